@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Attention forward+backward throughput on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole path over one batch: csa_attn_fwd (segment bounds / RoPE
+table, QK-norm+RoPE prologue, flash forward) then csa_attn_bwd (prologue recompute,
+delta preprocess, flash backward, dQ finalize), inputs resident in HBM.  The default
+workload is the 181M-model GQA shape (B=16, T=2048, 8 query / 4 KV heads, head dim 96,
+RoPE, QK-norm), the largest of the five shapes.  FLOPs are algorithmic: only the
+(query, key) pairs the mask keeps count, 4*D per pair per head forward, 10*D backward.
+
+Timing: W warm-up steps, then K steps, each bracketed by CUDA events on the launch stream
+with an L2 flush (256 MiB write) between steps outside the events; a barrier and a
+device synchronize on both sides; the max over ranks.  With N > 1 every rank runs its own
+batch (independent problems, weak scaling); the only collective is the timing reduction.
+`--impl reference` times the fp64 CPU oracle (the reference arm) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_self_attention_gqa_b200.workloads import BY_NAME, WORKLOADS, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = WORKLOADS[3].name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def visible_pairs(w, segment_ids) -> int:
+    """Number of unmasked (query, key) pairs summed over batch rows, per head."""
+    T, W = w.T, w.window
+    total = 0
+    for b in range(w.B):
+        if segment_ids is not None:
+            ids = np.asarray(segment_ids[b])
+            starts = np.concatenate([[0], np.nonzero(np.diff(ids))[0] + 1])
+            ends = np.concatenate([starts[1:], [T]])
+        else:
+            starts, ends = np.array([0]), np.array([T])
+        for s, e in zip(starts, ends):
+            L = int(e - s)
+            i = np.arange(L)
+            if w.causal:
+                cnt = i + 1
+                if W > 0:
+                    cnt = np.minimum(cnt, W)
+            else:
+                lo = np.maximum(0, i - W + 1) if W > 0 else np.zeros_like(i)
+                hi = np.minimum(L - 1, i + W - 1) if W > 0 else np.full_like(i, L - 1)
+                cnt = hi - lo + 1
+            total += int(cnt.sum())
+    return total
+
+
+def flops(w, segment_ids):
+    pairs = visible_pairs(w, segment_ids)
+    fwd = 4.0 * w.Hq * w.D * pairs
+    bwd = 10.0 * w.Hq * w.D * pairs
+    return fwd, bwd, pairs
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured (MEASURED_PEAKS.json)"
+    return FALLBACK_PEAKS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel source is
+    unchanged since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                a, b = line.strip().split("=", 1)
+                kv[a.strip()] = b.strip()
+    src = os.path.join(ROOT, "causal_self_attention_gqa_b200", "csrc", kv.get("source", ""))
+    if not os.path.exists(src) or "source_sha256" not in kv:
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != kv["source_sha256"]:
+            return None
+    try:
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark(self, which):
+        if which == "begin":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append(dict(ts=ts, sm=float(parts[2]), smax=float(parts[3]), active=parts[5],
+                                     hw=parts[6], hwt=parts[7], swt=parts[8], pcap=parts[9]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"samples": 0}
+        inside = [r for r in rows if self.t0 - 0.05 <= r["ts"] <= self.t1 + 0.05] or rows
+        reasons = set()
+        for r in inside:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in inside), "sm_max_mhz": max(r["smax"] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside),
+                "samples_in_timed_region": sum(1 for r in rows if self.t0 <= r["ts"] <= self.t1)}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_sample(w, inp, step: int, threads: int):
+    """One bounded sample of the workload on the CPU oracle: one batch row and one
+    key/value head group (its G query heads), forward + backward."""
+    import oracle
+    oracle.build()
+    oracle.set_threads(threads)
+    G = w.Hq // w.Hkv
+    b = step % w.B
+    g = (step // w.B) % w.Hkv
+    sl = slice(b, b + 1)
+    q = inp["q"][sl, :, g * G:(g + 1) * G]
+    k = inp["k"][sl, :, g:g + 1]
+    v = inp["v"][sl, :, g:g + 1]
+    do = inp["do"][sl, :, g * G:(g + 1) * G]
+    seg = inp["segment_ids"][sl] if inp["segment_ids"] is not None else None
+    kw = w.options()
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, segment_ids=seg, **kw)
+    oracle.attn_bwd(q, k, v, do, segment_ids=seg, **kw)
+    dt = time.perf_counter() - t0
+    sub = w.with_(B=1, Hq=G, Hkv=1)
+    f, bw, _ = flops(sub, seg.numpy() if seg is not None else None)
+    return (f + bw) / dt / 1e12, dt, f + bw
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = make_inputs(w)
+    cores = len(os.sched_getaffinity(0))
+    threads = min(cores, w.Hq // w.Hkv)
+    for s in range(args.warmup):
+        oracle_sample(w, inp, s, threads)
+    times, fl = [], []
+    for s in range(args.steps):
+        _, dt, f = oracle_sample(w, inp, args.warmup + s, threads)
+        times.append(dt)
+        fl.append(f)
+    value = sum(fl) / sum(times) / 1e12
+    sample = (f"one batch row x one KV-head group ({w.Hq // w.Hkv} query heads) of {w.name} per step, "
+              f"fwd+bwd, fp64")
+    line = {"impl": "reference", "metric": metric_name(), "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def metric_name():
+    return "causal attn fwd+bwd TFLOP/s and tokens/s on 1 B200; % of dense BF16 peak"
+
+
+def config_dict(w, n):
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "options": {k: v for k, v in w.options().items()},
+            "packed_segments": None if w.seg_len is None else list(w.seg_len),
+            "global_batch": w.B * n, "seq_len": w.T, "parallelism": f"dp{n}" if n > 1 else "single",
+            "l2": "flushed between timed steps (256 MiB write, outside the events)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(BY_NAME))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end leg (default: min(K, 20))")
+    args = ap.parse_args()
+    w = BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from causal_self_attention_gqa_b200 import _binding as csa
+
+    # every rank runs its own batch of the workload (weak scaling)
+    wr = w.with_(seed=w.seed + 7919 * rank)
+    inp = make_inputs(wr)
+    seg_np = inp["segment_ids"].numpy() if inp["segment_ids"] is not None else None
+    f_fwd, f_bwd, pairs = flops(wr, seg_np)
+    kw = wr.options()
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    seg = inp["segment_ids"].to(dev) if inp["segment_ids"] is not None else None
+    ws = csa.workspace_for(q, k, True, **kw)
+    o = torch.empty_like(q)
+    lse = torch.empty((wr.B, wr.Hq, wr.T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.attn_fwd(q, k, v, segment_ids=seg, out=o, lse=lse, workspace=ws, **kw)
+        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {csa.status_string(rc)}")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    csa.timing_enable(True)
+    sampler.mark("begin")
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("end")
+    csa.timing_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    kt = csa.timing_collect()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"device status after the timed region: {csa.status_string(rc)}")
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    total_flops = (f_fwd + f_bwd) * world * args.steps
+    value = total_flops / (ms_max * 1e-3) / 1e12
+    tokens_per_s = wr.B * wr.T * world * args.steps / (ms_max * 1e-3)
+
+    # per-kernel times (library events on the launch stream, same timed region)
+    launches = sum(c for _, c in kt.values())
+    per_kernel = {name: {"ms_avg": (t / c if c else 0.0), "launches": c, "share": 0.0} for name, (t, c) in kt.items()}
+    tot_k = sum(t for t, _ in kt.values()) or 1.0
+    for name, (t, c) in kt.items():
+        per_kernel[name]["share"] = t / tot_k
+    fwd_ms = per_kernel["k_attn_fwd"]["ms_avg"]
+    bwd_ms = per_kernel["k_attn_bwd"]["ms_avg"]
+    dom = max(("k_attn_fwd", "k_attn_bwd"), key=lambda n: kt[n][0])
+    dom_flops = f_fwd if dom == "k_attn_fwd" else f_bwd
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = dom_flops / (per_kernel[dom]["ms_avg"] * 1e-3) / 1e12 if per_kernel[dom]["ms_avg"] > 0 else 0.0
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(dom, wr.name), "kernel": dom,
+                "peak_source": f"{peak_src}, bf16_tflops (burst cuBLAS GEMM)"}
+
+    # end-to-end through the public API from pinned host buffers (rank-local)
+    e2e = None
+    n_e2e = args.e2e_steps or min(args.steps, 20)
+    if n_e2e > 0:
+        hq, hk, hv, hdo = (inp[n].pin_memory() for n in ("q", "k", "v", "do"))
+        hseg = inp["segment_ids"].pin_memory() if inp["segment_ids"] is not None else None
+        ho, hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, dq, dk, dv))
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo)) + \
+            (hseg.numel() * 4 if hseg is not None else 0)
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            dq_, dk_, dv_ = (hq.to(dev, non_blocking=True), hk.to(dev, non_blocking=True),
+                             hv.to(dev, non_blocking=True))
+            ddo = hdo.to(dev, non_blocking=True)
+            dseg = hseg.to(dev, non_blocking=True) if hseg is not None else None
+            oo, ll = csa.attn_fwd(dq_, dk_, dv_, segment_ids=dseg, workspace=ws, **kw)
+            gq, gk, gv = csa.attn_bwd(dq_, dk_, dv_, oo, ddo, ll, segment_ids=dseg, workspace=ws, **kw)
+            ho.copy_(oo, non_blocking=True)
+            hlse.copy_(ll, non_blocking=True)
+            hdq.copy_(gq, non_blocking=True)
+            hdk.copy_(gk, non_blocking=True)
+            hdv.copy_(gv, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": (f_fwd + f_bwd) * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": e_ms / n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = len(os.sched_getaffinity(0))
+        threads = min(cores, wr.Hq // wr.Hkv)
+        val, dt, _ = oracle_sample(wr, inp, 0, threads)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"one batch row x one KV-head group ({wr.Hq // wr.Hkv} query heads) of {wr.name}, "
+                         f"fwd+bwd in fp64, {dt:.1f} s"}
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak_spec = 2250.0
+    line = {
+        "metric": metric_name(), "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see workloads.py)",
+        "config": config_dict(wr, world),
+        "tokens_per_s": tokens_per_s,
+        "pct_of_peak": {"measured_burst": 100.0 * value / world / peak, "spec_2250": 100.0 * value / world / peak_spec},
+        "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
+        "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
+        "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd, "pairs_per_head": pairs},
+        "kernels": per_kernel,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,378 @@
+// api.cu -- the C ABI of libcsa.so (declared in include/csa.h): argument validation,
+// workspace layout, TMA tensor maps, kernel launches and optional per-kernel timing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "csa_internal.h"
+
+namespace csa {
+cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end, float2* rope_cs,
+                        double rope_base, cudaStream_t st);
+cudaError_t launch_prologue(const Problem& P, const void* q, const void* k, void* qo, void* ko, cudaStream_t st);
+cudaError_t launch_bwd_pre(const Problem& P, const void* o, const void* dout, float* delta, float* dq_acc,
+                           cudaStream_t st);
+cudaError_t launch_dq_finalize(const Problem& P, const float* dq_acc, const void* q, void* dq, cudaStream_t st);
+cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                       float* lse, cudaStream_t st);
+cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
+                       void* dk, void* dv, cudaStream_t st);
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ------------------------------------------------------------------ workspace layout
+struct Layout {
+    size_t status = 0, seg_start = 0, seg_end = 0, rope = 0, qp = 0, kp = 0, delta = 0, dq_acc = 0, total = 0;
+};
+
+bool needs_prologue(const csa_params& p) { return p.qk_norm != 0 || p.rope_base > 0.f; }
+
+Layout layout(const csa_params& p, bool backward, bool has_seg) {
+    Layout L;
+    const size_t BT = (size_t)p.B * p.T;
+    size_t off = 0;
+    L.status = off;
+    off += kAlign;
+    if (has_seg) {
+        L.seg_start = off;
+        off += up(BT * 4);
+        L.seg_end = off;
+        off += up(BT * 4);
+    }
+    if (p.rope_base > 0.f) {
+        L.rope = off;
+        off += up((size_t)p.T * (p.D / 2) * 8);
+    }
+    if (needs_prologue(p)) {
+        L.qp = off;
+        off += up(BT * p.Hq * p.D * 2);
+        L.kp = off;
+        off += up(BT * p.Hkv * p.D * 2);
+    }
+    if (backward) {
+        L.delta = off;
+        off += up(BT * p.Hq * 4);
+        L.dq_acc = off;
+        off += up(BT * p.Hq * p.D * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+int check_params(const csa_params* p) {
+    if (!p) return CSA_ERR_INVALID_ARG;
+    if (p->B < 0 || p->T < 0 || p->T > (1 << 20)) return CSA_ERR_INVALID_ARG;
+    if (p->Hq < 1 || p->Hkv < 1 || p->Hq % p->Hkv != 0) return CSA_ERR_INVALID_ARG;
+    if (p->D != 32 && p->D != 64 && p->D != 96 && p->D != 128) return CSA_ERR_INVALID_ARG;
+    if (p->causal != 0 && p->causal != 1) return CSA_ERR_INVALID_ARG;
+    if (!isfinite(p->softcap) || !isfinite(p->rope_base) || !isfinite(p->scale)) return CSA_ERR_INVALID_ARG;
+    if (p->qk_norm != 0 && p->qk_norm != 1) return CSA_ERR_INVALID_ARG;
+    if (p->qk_norm && !(p->qk_norm_eps > 0.f && isfinite(p->qk_norm_eps))) return CSA_ERR_INVALID_ARG;
+    const double elems = (double)p->B * p->T * p->Hq * p->D;
+    if (elems * 4.0 > 9.0e18) return CSA_ERR_INVALID_ARG;
+    return CSA_OK;
+}
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+// ------------------------------------------------------------------ device checks
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    static int known[64] = {0};  // 0 unknown, 1 ok, 2 wrong arch
+    if (dev < 64 && known[dev]) return known[dev] == 1 ? CSA_OK : CSA_ERR_ARCH;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    const bool ok = (major == 10 && minor == 0);
+    if (dev < 64) known[dev] = ok ? 1 : 2;
+    return ok ? CSA_OK : CSA_ERR_ARCH;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// [B, T, H, D] bf16 tensor, boxes of (swizzle-atom width) x 1 head x 128 rows x 1 batch.
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int sw = (D % 64 == 0) ? 128 : 64;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {(cuuint32_t)(sw / 2), 1, (cuuint32_t)kBM, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ timing
+struct TimingRec {
+    int kernel;
+    cudaEvent_t a, b;
+};
+bool g_timing = false;
+std::vector<TimingRec> g_records;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return e;
+}
+
+template <class F>
+int timed(int kernel, cudaStream_t st, F&& launch) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (g_timing) {
+        a = take_event();
+        b = take_event();
+        if (a) cudaEventRecord(a, st);
+    }
+    const cudaError_t e = launch();
+    if (g_timing && a && b) {
+        cudaEventRecord(b, st);
+        g_records.push_back({kernel, a, b});
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_LAUNCH;
+    }
+    return CSA_OK;
+}
+
+Problem make_problem(const csa_params& p, int* status) {
+    Problem P;
+    P.B = p.B;
+    P.T = p.T;
+    P.Hq = p.Hq;
+    P.Hkv = p.Hkv;
+    P.D = p.D;
+    P.G = p.Hq / p.Hkv;
+    P.causal = p.causal;
+    P.window = p.window > 0 ? p.window : 0;
+    P.softcap = p.softcap > 0.f ? p.softcap : 0.f;
+    P.scale = p.scale > 0.f ? p.scale : (float)(1.0 / sqrt((double)p.D));
+    P.scale_log2 = (float)((double)P.scale * 1.4426950408889634);
+    P.rope = p.rope_base > 0.f ? 1 : 0;
+    P.qk_norm = p.qk_norm;
+    P.eps = p.qk_norm_eps;
+    P.seg_start = nullptr;
+    P.seg_end = nullptr;
+    P.rope_cs = nullptr;
+    P.status = status;
+    return P;
+}
+
+// Shared front half of both calls: checks, status reset, segments, RoPE table, prologue.
+struct Prepared {
+    Problem P;
+    Layout L;
+    const void* qk_q;  // tensors the attention kernels read as Q and K (raw or prologue output)
+    const void* qk_k;
+};
+
+int prepare(const csa_params* p, bool backward, const void* q, const void* k, const int32_t* seg, void* ws,
+            size_t ws_bytes, cudaStream_t st, Prepared& out) {
+    const bool has_seg = seg != nullptr;
+    out.L = layout(*p, backward, has_seg);
+    if (ws_bytes < out.L.total) return CSA_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    out.P = make_problem(*p, reinterpret_cast<int*>(w + out.L.status));
+    if (cudaMemsetAsync(w + out.L.status, 0, sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    int32_t* ss = has_seg ? reinterpret_cast<int32_t*>(w + out.L.seg_start) : nullptr;
+    int32_t* se = has_seg ? reinterpret_cast<int32_t*>(w + out.L.seg_end) : nullptr;
+    float2* rope = p->rope_base > 0.f ? reinterpret_cast<float2*>(w + out.L.rope) : nullptr;
+    out.P.seg_start = ss;
+    out.P.seg_end = se;
+    out.P.rope_cs = rope;
+    if (has_seg || rope) {
+        const int rc = timed(kPrep, st, [&] { return launch_prep(out.P, seg, ss, se, rope, p->rope_base, st); });
+        if (rc) return rc;
+    }
+    out.qk_q = q;
+    out.qk_k = k;
+    if (needs_prologue(*p)) {
+        void* qp = w + out.L.qp;
+        void* kp = w + out.L.kp;
+        const int rc = timed(kPrologue, st, [&] { return launch_prologue(out.P, q, k, qp, kp, st); });
+        if (rc) return rc;
+        out.qk_q = qp;
+        out.qk_k = kp;
+    }
+    return CSA_OK;
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+size_t csa_workspace_size(const csa_params* p, int for_backward) {
+    if (check_params(p) != CSA_OK) return 0;
+    // segment_ids may or may not be passed: size for the larger case
+    return layout(*p, for_backward != 0, true).total;
+}
+
+int csa_attn_fwd(const csa_params* p, const void* q, const void* k, const void* v, const int32_t* segment_ids, void* o,
+                 float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (p->B == 0 || p->T == 0) return CSA_OK;
+    if (!q || !k || !v || !o || !lse || !workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(workspace, 256) || (segment_ids && !aligned(segment_ids, 4)))
+        return CSA_ERR_ALIGNMENT;
+    if (workspace_bytes < layout(*p, false, segment_ids != nullptr).total) return CSA_ERR_WORKSPACE;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Prepared pr;
+    if ((rc = prepare(p, false, q, k, segment_ids, workspace, workspace_bytes, st, pr))) return rc;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D))
+        return CSA_ERR_CUDA;
+    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, o, lse, st); });
+}
+
+int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, const int32_t* segment_ids, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (p->B == 0 || p->T == 0) return CSA_OK;
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(workspace, 256) ||
+        (segment_ids && !aligned(segment_ids, 4)))
+        return CSA_ERR_ALIGNMENT;
+    if (workspace_bytes < layout(*p, true, segment_ids != nullptr).total) return CSA_ERR_WORKSPACE;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Prepared pr;
+    if ((rc = prepare(p, true, q, k, segment_ids, workspace, workspace_bytes, st, pr))) return rc;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    float* delta = reinterpret_cast<float*>(w + pr.L.delta);
+    float* dq_acc = reinterpret_cast<float*>(w + pr.L.dq_acc);
+    if ((rc = timed(kBwdPre, st, [&] { return launch_bwd_pre(pr.P, o, dout, delta, dq_acc, st); }))) return rc;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&tdo, dout, p->B, p->T, p->Hq, p->D))
+        return CSA_ERR_CUDA;
+    if ((rc = timed(kBwd, st,
+                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, lse, delta, dq_acc, k, dk, dv, st); })))
+        return rc;
+    return timed(kDqFinalize, st, [&] { return launch_dq_finalize(pr.P, dq_acc, q, dq, st); });
+}
+
+int csa_device_status(void* workspace, void* stream) {
+    if (!workspace) return CSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    int code = 0;
+    if (cudaMemcpy(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    if (code != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    return code;
+}
+
+const char* csa_status_string(int code) {
+    switch (code) {
+        case CSA_OK: return "ok";
+        case CSA_ERR_INVALID_ARG: return "invalid argument (shape, head ratio, head dim, option or null pointer)";
+        case CSA_ERR_ALIGNMENT: return "misaligned pointer (tensors need 16 bytes, workspace 256 bytes)";
+        case CSA_ERR_WORKSPACE: return "workspace smaller than csa_workspace_size()";
+        case CSA_ERR_ARCH: return "device is not a compute capability 10.0 (B200) GPU";
+        case CSA_ERR_LAUNCH: return "kernel launch failed";
+        case CSA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel ran out";
+        case CSA_ERR_CUDA: return "CUDA runtime or driver call failed";
+        case CSA_ERR_NOT_IMPLEMENTED: return "not implemented";
+        default: return "unknown status code";
+    }
+}
+
+int csa_timing_enable(int enable) {
+    g_timing = enable != 0;
+    return CSA_OK;
+}
+
+int csa_timing_collect(double* total_ms, int* launches, int n) {
+    int rc = CSA_OK;
+    for (const TimingRec& r : g_records) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+            cudaGetLastError();
+            rc = CSA_ERR_CUDA;
+        } else if (r.kernel < n) {
+            if (total_ms) total_ms[r.kernel] += ms;
+            if (launches) launches[r.kernel] += 1;
+        }
+        g_event_pool.push_back(r.a);
+        g_event_pool.push_back(r.b);
+    }
+    g_records.clear();
+    return rc;
+}
+
+int csa_num_kernels(void) { return kNumKernels; }
+
+const char* csa_kernel_name(int k) {
+    static const char* names[kNumKernels] = {"k_prep", "k_qk_prologue", "k_attn_fwd",
+                                             "k_bwd_pre", "k_attn_bwd", "k_dq_finalize"};
+    return (k >= 0 && k < kNumKernels) ? names[k] : "";
+}
+
+}  // extern "C"

@@ -1,0 +1,512 @@
+// attn_bwd.cu -- flash-style attention backward for sm_100a (TMA + tcgen05/TMEM).
+//
+// The gradient of the attention of attn_fwd.cu (the pages obtain it by automatic
+// differentiation of the same graph).  With P_ij = exp(s'_ij - LSE_i) recomputed from the
+// forward's log-sum-exp, dP_ij = dO_i . v_j and delta_i = sum_d dO_id O_id:
+//     dV_j  += sum_i P_ij dO_i
+//     dS_ij  = P_ij (dP_ij - delta_i) * (1 - tanh^2(s_ij / c))      (last factor: cap only)
+//     dQ'_i += scale sum_j dS_ij k'_j        dK'_j += scale sum_i dS_ij q'_i
+// followed by the transposed RoPE and RMSNorm on dK' (epilogue here) and dQ' (k_dq_finalize).
+//
+// One CTA owns a 128-key tile of one (b, kv head) and loops over the G query heads of the
+// group and every 128-row query tile that sees those keys, so dK and dV of the group sum in
+// TMEM without atomics.  dQ' tiles are added into an fp32 accumulator with vector reductions.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: K', V once; Q', dO tiles into a 2-stage ring
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 4-7   P / dS computation (thread = key row = TMEM lane), then the dK/dV epilogue
+//   warps 8-11  dQ' drain: TMEM -> fp32 reductions into the global accumulator
+// TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
+// written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
+// reuses the dP^T columns once dS has been formed.  dS^T goes to shared memory (128x128
+// bf16, 128-byte swizzle) where it is the K-major A operand of dK' and, read MN-major,
+// the A operand of dQ'.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "csa_internal.h"
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace csa {
+
+template <int D>
+struct BwdCfg {
+    static constexpr int SW = (D % 64 == 0) ? 128 : 64;
+    static constexpr int AE = SW / 2;
+    static constexpr int NA = D / AE;
+    static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
+    static constexpr int TILE = kBM * D * 2;
+    static constexpr int STAGES = 2;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = TILE;
+    static constexpr int OFF_Q = 2 * TILE;
+    static constexpr int OFF_DO = OFF_Q + STAGES * TILE;
+    static constexpr int OFF_DS = OFF_DO + STAGES * TILE;    // 128 x 128 bf16, SW128
+    static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;   // 2 x 128 fp32 (log2 units)
+    static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
+    static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
+    // kv_full, q_full[2], do_full[2], stage_empty[2], s_full, dp_full, ds_full, ds_free,
+    // dq_full, dq_empty, acc_full, wg_sync
+    static constexpr int NBAR = 15;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+    static constexpr uint32_t IDESC_KV = idesc_bf16(128, D, false, true);    // dV, dK
+    static constexpr uint32_t IDESC_Q = idesc_bf16(128, D, true, true);      // dQ'
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+struct BwdArgs {
+    Problem P;
+    const float* lse;      // [B, Hq, T] natural log
+    const float* delta;    // [B, Hq, T]
+    float* dq_acc;         // [B, T, Hq, D] fp32, zeroed
+    const __nv_bfloat16* k_raw;  // raw K (for the RMSNorm backward of dK)
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    int nkt;  // key tiles per (b, kv head)
+};
+
+template <int D>
+__device__ __forceinline__ uint64_t bdesc_kmajor(uint32_t tile, int ks) {
+    using C = BwdCfg<D>;
+    const int e = ks * 16;
+    return sdesc(tile + (e / C::AE) * (kBM * C::SW) + (e % C::AE) * 2, 16, 8 * C::SW, C::LAYOUT);
+}
+template <int D>
+__device__ __forceinline__ uint64_t bdesc_mnmajor(uint32_t tile, int ks) {
+    using C = BwdCfg<D>;
+    return sdesc(tile + ks * 16 * C::SW, kBM * C::SW, 8 * C::SW, C::LAYOUT);
+}
+// dS^T tile: 128 key rows x 128 query columns, 128-byte swizzle, two 64-column atoms.
+__device__ __forceinline__ uint64_t ds_desc_kmajor(uint32_t tile, int ks) {  // A of dK: M = key, K = q
+    const int e = ks * 16;
+    return sdesc(tile + (e / 64) * (128 * 128) + (e % 64) * 2, 16, 1024, kLayoutSw128);
+}
+__device__ __forceinline__ uint64_t ds_desc_mnmajor(uint32_t tile, int ks) {  // A of dQ: M = q, K = key
+    return sdesc(tile + ks * 16 * 128, 128 * 128, 1024, kLayoutSw128);
+}
+
+// Queries that see key j: [lo, hi] (empty when lo > hi).
+__device__ __forceinline__ void col_bounds(const Problem& P, int b, int j, int& lo, int& hi) {
+    if (j >= P.T || j < 0) {
+        lo = P.T;
+        hi = -1;
+        return;
+    }
+    int l = P.causal ? j : 0, h = P.T - 1;
+    if (P.seg_start) {
+        l = max(l, (int)P.seg_start[(size_t)b * P.T + j]);
+        h = min(h, P.seg_end[(size_t)b * P.T + j] - 1);
+    }
+    if (P.window > 0) {
+        h = min(h, j + P.window - 1);
+        if (!P.causal) l = max(l, j - P.window + 1);
+    }
+    lo = l;
+    hi = h;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const BwdArgs A) {
+    using C = BwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const Problem& P = A.P;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* q_full = bars + 1;       // [2]
+    uint64_t* do_full = bars + 3;      // [2]
+    uint64_t* stage_empty = bars + 5;  // [2]
+    uint64_t* s_full = bars + 7;
+    uint64_t* dp_full = bars + 8;
+    uint64_t* ds_full = bars + 9;
+    uint64_t* ds_free = bars + 10;
+    uint64_t* dq_full = bars + 11;
+    uint64_t* dq_empty = bars + 12;
+    uint64_t* acc_full = bars + 13;
+    uint64_t* wg_sync = bars + 14;  // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
+    float* delta_s = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+
+    // ---- work item: key tile n of (b, kvh); heavy (small n, causal) first
+    const int n = blockIdx.x / (P.B * P.Hkv);
+    const int b = (blockIdx.x % (P.B * P.Hkv)) / P.Hkv;
+    const int kvh = blockIdx.x % P.Hkv;
+    int m_lo, m_hi;
+    {
+        int lo0, hi0, lo1, hi1;
+        col_bounds(P, b, n * kBN, lo0, hi0);
+        col_bounds(P, b, min(n * kBN + kBN - 1, P.T - 1), lo1, hi1);
+        m_lo = lo0 / kBM;
+        m_hi = hi1 / kBM;
+    }
+    const int nm = m_hi - m_lo + 1;
+    const int nit = nm > 0 ? P.G * nm : 0;
+
+    // the swizzled tiles need a 1024-byte aligned base; the condition is uniform over the CTA
+    if ((smem_u32(smem) & 1023u) != 0) {
+        if (tid == 0) atomicCAS(P.status, 0, CSA_ERR_LAUNCH);
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&do_full[s], 1);
+            mbar_init(&stage_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(ds_free, 1);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_empty, 128);
+        mbar_init(acc_full, 1);
+        mbar_init(wg_sync, 128);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= TMA producer
+        if (lane == 0 && nit > 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_do);
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+            for (int a = 0; a < C::NA; ++a) {
+                tma_load_4d(&tm_k, kv_full, smem + C::OFF_K + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
+                tma_load_4d(&tm_v, kv_full, smem + C::OFF_V + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
+            }
+            for (int it = 0; it < nit; ++it) {
+                const int s = it & 1;
+                if (it >= 2 && !mbar_wait(&stage_empty[s], ((it >> 1) - 1) & 1, abort_flag, P.status)) break;
+                const int h = kvh * P.G + it / nm;
+                const int m = m_lo + it % nm;
+                mbar_arrive_expect_tx(&q_full[s], C::TILE);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_q, &q_full[s], smem + C::OFF_Q + s * C::TILE + a * kBM * C::SW, a * C::AE, h,
+                                m * kBM, b);
+                mbar_arrive_expect_tx(&do_full[s], C::TILE);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_do, &do_full[s], smem + C::OFF_DO + s * C::TILE + a * kBM * C::SW, a * C::AE, h,
+                                m * kBM, b);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0 && nit > 0) {
+            const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
+            const uint32_t sq = smem_u32(smem + C::OFF_Q), sdo = smem_u32(smem + C::OFF_DO);
+            const uint32_t sds = smem_u32(smem + C::OFF_DS);
+            const uint32_t t_dv = tmem, t_dk = tmem + 128, t_s = tmem + 256, t_dp = tmem + 384;
+            bool ok = mbar_wait(kv_full, 0, abort_flag, P.status);
+            for (int it = 0; ok && it < nit; ++it) {
+                const int s = it & 1, ph = (it >> 1) & 1;
+                if (!(ok = mbar_wait(&q_full[s], ph, abort_flag, P.status))) break;
+                tc_fence_after();
+                // S^T = K' Q'^T  (M = 128 keys, N = 128 queries, K = D)
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_ss(t_s, bdesc_kmajor<D>(sk, ks), bdesc_kmajor<D>(sq + s * C::TILE, ks), C::IDESC_S, ks > 0);
+                umma_commit(s_full);
+                if (!(ok = mbar_wait(&do_full[s], ph, abort_flag, P.status))) break;
+                if (it > 0 && !(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, P.status))) break;
+                tc_fence_after();
+                // dP^T = V dO^T
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_ss(t_dp, bdesc_kmajor<D>(sv, ks), bdesc_kmajor<D>(sdo + s * C::TILE, ks), C::IDESC_S, ks > 0);
+                umma_commit(dp_full);
+                if (!(ok = mbar_wait(ds_full, it & 1, abort_flag, P.status))) break;
+                tc_fence_after();
+                // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
+#pragma unroll
+                for (int ks = 0; ks < kBM / 16; ++ks)
+                    umma_ts(t_dv, t_s + ks * 8, bdesc_mnmajor<D>(sdo + s * C::TILE, ks), C::IDESC_KV,
+                            (it > 0 || ks > 0) ? 1u : 0u);
+                // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
+#pragma unroll
+                for (int ks = 0; ks < kBM / 16; ++ks)
+                    umma_ss(t_dk, ds_desc_kmajor(sds, ks), bdesc_mnmajor<D>(sq + s * C::TILE, ks), C::IDESC_KV,
+                            (it > 0 || ks > 0) ? 1u : 0u);
+                // dQ' = dS K'  (A = dS, MN-major view of the same tile; B = K', MN-major)
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    umma_ss(t_dp, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
+                umma_commit(dq_full);
+                umma_commit(&stage_empty[s]);
+                umma_commit(ds_free);
+            }
+            if (ok) umma_commit(acc_full);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ================= P / dS, then the dK / dV epilogue
+        const int kr = tid - 128;
+        const int key = n * kBN + kr;
+        int lo, hi;
+        col_bounds(P, b, key, lo, hi);
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + 256, t_dp = tmem + lane_base + 384;
+        uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
+        const float kLog2e = 1.4426950408889634f;
+        bool ok = nit > 0;
+        for (int it = 0; ok && it < nit; ++it) {
+            const int h = kvh * P.G + it / nm;
+            const int m = m_lo + it % nm;
+            const int q0 = m * kBM;
+            const int buf = it & 1;
+            {
+                const int q = q0 + kr;
+                const size_t o = ((size_t)b * P.Hq + h) * P.T + q;
+                lse_s[buf * 128 + kr] = (q < P.T) ? A.lse[o] * kLog2e : INFINITY;
+                delta_s[buf * 128 + kr] = (q < P.T) ? A.delta[o] : 0.f;
+            }
+            mbar_arrive(wg_sync);
+            ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
+            ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status) &&
+                 mbar_wait(dp_full, it & 1, abort_flag, P.status);
+            if (ok && it > 0) ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const bool full = (q0 >= lo) && (q0 + kBM - 1 <= hi);
+            const float* ls = lse_s + buf * 128;
+            const float* dl = delta_s + buf * 128;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dpv[32];
+                tmem_ld32(t_s + 32 * c, sv);
+                tmem_ld32(t_dp + 32 * c, dpv);
+                tmem_ld_wait();
+                tmem_ld_fence(sv);
+                tmem_ld_fence(dpv);
+                uint32_t pk[16], dk16[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float pp[2], dd[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int qi = 32 * c + e + u;
+                        const float raw = __uint_as_float(sv[e + u]);
+                        float x, dfac = 1.f;
+                        if (P.softcap > 0.f) {
+                            const float y = raw * P.scale / P.softcap;
+                            const float ex = ex2(y * 2.8853900817779268f);
+                            const float t = 1.0f - __fdividef(2.0f, ex + 1.0f);
+                            x = P.softcap * kLog2e * t;
+                            dfac = 1.0f - t * t;
+                        } else {
+                            x = raw * P.scale_log2;
+                        }
+                        float p = ex2(x - ls[qi]);
+                        if (!full) {
+                            const int q = q0 + qi;
+                            if (q < lo || q > hi) p = 0.f;
+                        }
+                        pp[u] = p;
+                        dd[u] = p * (__uint_as_float(dpv[e + u]) - dl[qi]) * dfac;
+                    }
+                    pk[e / 2] = pack_bf16x2(pp[0], pp[1]);
+                    dk16[e / 2] = pack_bf16x2(dd[0], dd[1]);
+                }
+                tmem_st16(t_s + 16 * c, pk);  // P^T (bf16) over S^T columns already read
+                // dS^T row kr, queries [32c, 32c+32): 4 chunks of 16 bytes, 128-byte swizzle
+                uint8_t* atom_row = ds_row + (c >> 1) * (128 * 128);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    const int chunk = ((c & 1) * 4 + v4) ^ (kr & 7);
+                    *reinterpret_cast<uint4*>(atom_row + chunk * 16) =
+                        make_uint4(dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
+                }
+            }
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        // ---- epilogue: dV, dK of this key row (sum over the group's query heads)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, P.status));
+        if (ok) {
+            tc_fence_after();
+            const bool row_ok = key < P.T;
+            const size_t row_off = (((size_t)b * P.T + (row_ok ? key : 0)) * P.Hkv + kvh) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + 32 * c, v);
+                tmem_ld_wait();
+                tmem_ld_fence(v);
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(A.dv + row_off + 32 * c);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * v4]), __uint_as_float(v[8 * v4 + 1])),
+                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3])),
+                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5])),
+                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7])));
+                }
+            }
+            // dK = RMSNorm^T(RoPE^T(scale * dK')), two passes over 16-pair chunks (lo, hi halves)
+            const uint32_t t_dk = tmem + lane_base + 128;
+            constexpr int kHalf = D / 2;
+            const int pos = row_ok ? (P.seg_start ? key - P.seg_start[(size_t)b * P.T + key] : key) : 0;
+            const __nv_bfloat16* xr = A.k_raw + row_off;
+            float ss = 0.f, dot = 0.f;
+            if (P.qk_norm) {
+#pragma unroll 1
+                for (int c = 0; c < kHalf / 16; ++c) {
+                    uint32_t ulo[16], uhi[16];
+                    tmem_ld16(t_dk + 16 * c, ulo);
+                    tmem_ld16(t_dk + kHalf + 16 * c, uhi);
+                    tmem_ld_wait();
+                    tmem_ld_fence(ulo);
+                    tmem_ld_fence(uhi);
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4) {
+                        float xl[4] = {0.f, 0.f, 0.f, 0.f}, xh[4] = {0.f, 0.f, 0.f, 0.f};
+                        if (row_ok) {
+                            load_bf16x4(xr + 16 * c + e, xl);
+                            load_bf16x4(xr + kHalf + 16 * c + e, xh);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            float ga = __uint_as_float(ulo[e + u]) * P.scale;
+                            float gb = __uint_as_float(uhi[e + u]) * P.scale;
+                            if (P.rope) rope_transpose(ga, gb, P.rope_cs[(size_t)pos * kHalf + 16 * c + e + u]);
+                            ss += xl[u] * xl[u] + xh[u] * xh[u];
+                            dot += ga * xl[u] + gb * xh[u];
+                        }
+                    }
+                }
+            }
+            const float rs = P.qk_norm ? 1.0f / sqrtf(ss / (float)D + P.eps) : 1.f;
+            const float k3 = P.qk_norm ? rs * rs * rs * dot / (float)D : 0.f;
+#pragma unroll 1
+            for (int c = 0; c < kHalf / 16; ++c) {
+                uint32_t ulo[16], uhi[16];
+                tmem_ld16(t_dk + 16 * c, ulo);
+                tmem_ld16(t_dk + kHalf + 16 * c, uhi);
+                tmem_ld_wait();
+                tmem_ld_fence(ulo);
+                tmem_ld_fence(uhi);
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    float xl[4] = {0.f, 0.f, 0.f, 0.f}, xh[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (row_ok && P.qk_norm) {
+                        load_bf16x4(xr + 16 * c + e, xl);
+                        load_bf16x4(xr + kHalf + 16 * c + e, xh);
+                    }
+                    float ol[4], oh[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        float ga = __uint_as_float(ulo[e + u]) * P.scale;
+                        float gb = __uint_as_float(uhi[e + u]) * P.scale;
+                        if (P.rope) rope_transpose(ga, gb, P.rope_cs[(size_t)pos * kHalf + 16 * c + e + u]);
+                        ol[u] = rs * ga - k3 * xl[u];
+                        oh[u] = rs * gb - k3 * xh[u];
+                    }
+                    if (row_ok) {
+                        store_bf16x4(A.dk + row_off + 16 * c + e, ol);
+                        store_bf16x4(A.dk + row_off + kHalf + 16 * c + e, oh);
+                    }
+                }
+            }
+        }
+    } else if (warp >= 8) {
+        // ================= dQ' drain (thread = query row of the current tile)
+        const int r = tid - 256;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_dq = tmem + lane_base + 384;
+        bool ok = nit > 0;
+        for (int it = 0; ok && it < nit; ++it) {
+            const int h = kvh * P.G + it / nm;
+            const int q = (m_lo + it % nm) * kBM + r;
+            ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
+            if (!ok) break;
+            tc_fence_after();
+            float* dst = A.dq_acc + (((size_t)b * P.T + (q < P.T ? q : 0)) * P.Hq + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(t_dq + 32 * c, v);
+                tmem_ld_wait();
+                tmem_ld_fence(v);
+                if (q < P.T) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        red_add_v4(dst + 32 * c + 4 * v4, __uint_as_float(v[4 * v4]) * P.scale,
+                                   __uint_as_float(v[4 * v4 + 1]) * P.scale, __uint_as_float(v[4 * v4 + 2]) * P.scale,
+                                   __uint_as_float(v[4 * v4 + 3]) * P.scale);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dq_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc,
+                                const void* k_raw, void* dk, void* dv, cudaStream_t st) {
+    using C = BwdCfg<D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    BwdArgs A;
+    A.P = P;
+    A.lse = lse;
+    A.delta = delta;
+    A.dq_acc = dq_acc;
+    A.k_raw = static_cast<const __nv_bfloat16*>(k_raw);
+    A.dk = static_cast<__nv_bfloat16*>(dk);
+    A.dv = static_cast<__nv_bfloat16*>(dv);
+    A.nkt = (P.T + kBN - 1) / kBN;
+    const int grid = A.nkt * P.B * P.Hkv;
+    k_attn_bwd<D><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, A);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
+                       void* dk, void* dv, cudaStream_t st) {
+    switch (P.D) {
+        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace csa

@@ -1,0 +1,435 @@
+// attn_fwd.cu -- flash-style attention forward for sm_100a (TMA + tcgen05/TMEM).
+//
+// Computes, per (b, h) and query row i, O_i = sum_j softmax_j(s'_ij) v_j over the keys j
+// visible to i, and LSE_i = log sum_j exp(s'_ij) (natural log), where s'_ij is the scaled
+// (and optionally soft-capped) score of q'_i and k'_j: the scaled dot-product attention of
+// the GPT-pretraining page ("Multihead Attention"), with the grouped-query heads and
+// score soft-capping of the nanogpt-jax-181m model card ("Architecture").  The softmax is
+// evaluated online over key tiles (running max and sum, rescaling the partial output),
+// which reaches the same result as the row softmax up to rounding.
+//
+// One CTA owns up to two 128-row query tiles that read the same key/value head:
+//   * G = Hq/Hkv >= 2: two query heads of one group at the same 128 positions, so both
+//     tiles see exactly the same keys and share every K/V tile;
+//   * G == 1: two consecutive 128-position tiles of one head.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: the two Q tiles once, then K and V tiles into a STAGES ring
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 4-7   softmax of query tile 0 (thread = row = TMEM lane)
+//   warps 8-11  softmax of query tile 1
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).  P_i is
+// written as packed bf16 over the first 64 columns of S_i and fed to the PV MMA from TMEM.
+// MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one softmax group
+// works on its scores the tensor core serves the other one.
+// All mbarrier waits are bounded (see mbar_wait); a wait that runs out records
+// CSA_ERR_DEVICE_TIMEOUT and every role unwinds, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "csa_internal.h"
+#include "ptx.cuh"
+
+namespace csa {
+
+template <int D>
+struct FwdCfg {
+    static constexpr int SW = (D % 64 == 0) ? 128 : 64;  // swizzle span (bytes) of a tile row
+    static constexpr int AE = SW / 2;                     // bf16 elements per swizzle row
+    static constexpr int NA = D / AE;                     // swizzle-atom columns per tile
+    static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
+    static constexpr int TILE = kBM * D * 2;              // bytes of one 128 x D bf16 tile
+    static constexpr int STAGES = (D == 128) ? 2 : ((D == 96) ? 3 : 4);
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + STAGES * TILE;
+    static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+    // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2]
+    static constexpr int NBAR = 1 + 3 * STAGES + 6;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
+    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+    static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(D % AE == 0 && D % 32 == 0, "head dim");
+};
+
+struct FwdArgs {
+    Problem P;
+    __nv_bfloat16* o;
+    float* lse;
+    int nqt;    // query tiles per (b, h)
+    int pairs;  // G >= 2: head pairs per group; G == 1: tile pairs per head
+};
+
+// K-major operand (rows x D, D contiguous), 16-element K step ks.
+template <int D>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int ks) {
+    using C = FwdCfg<D>;
+    const int e = ks * 16;
+    return sdesc(tile + (e / C::AE) * (kBM * C::SW) + (e % C::AE) * 2, 16, 8 * C::SW, C::LAYOUT);
+}
+// MN-major operand (rows = K index, D contiguous = N index), 16-row K step ks.
+template <int D>
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks) {
+    using C = FwdCfg<D>;
+    return sdesc(tile + ks * 16 * C::SW, kBM * C::SW, 8 * C::SW, C::LAYOUT);
+}
+
+// Keys visible to query row q: [lo, hi] (empty when lo > hi).
+__device__ __forceinline__ void row_bounds(const Problem& P, int b, int q, int& lo, int& hi) {
+    if (q >= P.T || q < 0) {
+        lo = P.T;
+        hi = -1;
+        return;
+    }
+    int l = 0, h = P.causal ? q : P.T - 1;
+    if (P.seg_start) {
+        l = P.seg_start[(size_t)b * P.T + q];
+        h = min(h, P.seg_end[(size_t)b * P.T + q] - 1);
+    }
+    if (P.window > 0) {
+        l = max(l, q - P.window + 1);
+        if (!P.causal) h = min(h, q + P.window - 1);
+    }
+    lo = l;
+    hi = h;
+}
+
+__device__ __forceinline__ float capped_log2(float raw, const Problem& P) {
+    // s' * log2(e) with s' = c * tanh(s / c), s = scale * raw; tanh(y) = 1 - 2 / (exp(2y) + 1)
+    const float y = raw * P.scale / P.softcap;
+    const float e = ex2(y * 2.8853900817779268f);  // exp(2y)
+    const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
+    return P.softcap * 1.4426950408889634f * t;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdArgs A) {
+    using C = FwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const Problem& P = A.P;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = bars + 1 + C::STAGES;
+    uint64_t* kv_empty = bars + 1 + 2 * C::STAGES;
+    uint64_t* s_full = bars + 1 + 3 * C::STAGES;
+    uint64_t* p_full = s_full + 2;
+    uint64_t* o_full = s_full + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    // ---- work item
+    int b, kvh, hh[2], mm[2];
+    {
+        const int idx = blockIdx.x;
+        if (P.G >= 2) {
+            const int per = P.B * P.Hkv * A.pairs;
+            const int m = A.nqt - 1 - idx / per;
+            int rem = idx % per;
+            b = rem / (P.Hkv * A.pairs);
+            rem %= P.Hkv * A.pairs;
+            kvh = rem / A.pairs;
+            const int pg = rem % A.pairs;
+            hh[0] = kvh * P.G + 2 * pg;
+            hh[1] = (2 * pg + 1 < P.G) ? hh[0] + 1 : -1;
+            mm[0] = mm[1] = m;
+        } else {
+            const int per = P.B * P.Hq;
+            const int pp = A.pairs - 1 - idx / per;
+            const int rem = idx % per;
+            b = rem / P.Hq;
+            kvh = rem % P.Hq;
+            hh[0] = hh[1] = kvh;
+            mm[0] = 2 * pp;
+            mm[1] = 2 * pp + 1;
+            if (mm[1] >= A.nqt) hh[1] = -1;
+        }
+    }
+    const bool two = hh[1] >= 0;
+    // key-tile range: union over the (one or two) query tiles; bounds are monotone in q
+    int kt_begin, kt_end;
+    {
+        int lo0, hi0, lo1, hi1;
+        row_bounds(P, b, mm[0] * kBM, lo0, hi0);
+        const int last = two ? mm[1] : mm[0];
+        row_bounds(P, b, min(last * kBM + kBM - 1, P.T - 1), lo1, hi1);
+        kt_begin = lo0 / kBN;
+        kt_end = hi1 / kBN;
+    }
+    const int nkt = kt_end - kt_begin + 1;
+
+    // ---- setup
+    // the swizzled tiles need a 1024-byte aligned base; the condition is uniform over the CTA
+    if ((smem_u32(smem) & 1023u) != 0) {
+        if (tid == 0) atomicCAS(P.status, 0, CSA_ERR_LAUNCH);
+        return;
+    }
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&o_full[i], 1);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================= TMA producer
+        if (lane == 0 && nkt > 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const uint32_t qbytes = (two ? 2 : 1) * C::TILE;
+            mbar_arrive_expect_tx(q_full, qbytes);
+            for (int i = 0; i < (two ? 2 : 1); ++i)
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_q, q_full, smem + C::OFF_Q + i * C::TILE + a * kBM * C::SW, a * C::AE, hh[i],
+                                mm[i] * kBM, b);
+            for (int jj = 0; jj < nkt; ++jj) {
+                const int s = jj % C::STAGES;
+                if (jj >= C::STAGES && !mbar_wait(&kv_empty[s], ((jj / C::STAGES) - 1) & 1, abort_flag, P.status))
+                    break;
+                const int t0 = (kt_begin + jj) * kBN;
+                mbar_arrive_expect_tx(&k_full[s], C::TILE);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_k, &k_full[s], smem + C::OFF_K + s * C::TILE + a * kBM * C::SW, a * C::AE, kvh,
+                                t0, b);
+                mbar_arrive_expect_tx(&v_full[s], C::TILE);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_v, &v_full[s], smem + C::OFF_V + s * C::TILE + a * kBM * C::SW, a * C::AE, kvh,
+                                t0, b);
+            }
+        }
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        if (lane == 0 && nkt > 0) {
+            const uint32_t sq = smem_u32(smem + C::OFF_Q);
+            const uint32_t sk = smem_u32(smem + C::OFF_K);
+            const uint32_t sv = smem_u32(smem + C::OFF_V);
+            auto issue_s = [&](int i, int s) {
+                const uint32_t d = tmem + i * 128;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_ss(d, desc_kmajor<D>(sq + i * C::TILE, ks), desc_kmajor<D>(sk + s * C::TILE, ks), C::IDESC_S,
+                            ks > 0);
+                umma_commit(&s_full[i]);
+            };
+            auto issue_pv = [&](int i, int s, bool acc) {
+                const uint32_t d = tmem + 256 + i * 128;
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    umma_ts(d, tmem + i * 128 + ks * 8, desc_mnmajor<D>(sv + s * C::TILE, ks), C::IDESC_PV,
+                            (acc || ks > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, P.status) && mbar_wait(&k_full[0], 0, abort_flag, P.status);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                if (two) issue_s(1, 0);
+            }
+            for (int jj = 0; ok && jj < nkt; ++jj) {
+                const int s = jj % C::STAGES, ph = (jj / C::STAGES) & 1;
+                const bool next = jj + 1 < nkt;
+                const int s2 = (jj + 1) % C::STAGES, ph2 = ((jj + 1) / C::STAGES) & 1;
+                ok = mbar_wait(&v_full[s], ph, abort_flag, P.status) && mbar_wait(&p_full[0], jj & 1, abort_flag, P.status);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(0, s, jj > 0);
+                if (next) {
+                    if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, P.status))) break;
+                    tc_fence_after();
+                    issue_s(0, s2);
+                }
+                if (two) {
+                    if (!(ok = mbar_wait(&p_full[1], jj & 1, abort_flag, P.status))) break;
+                    tc_fence_after();
+                    issue_pv(1, s, jj > 0);
+                    if (next) issue_s(1, s2);
+                }
+                umma_commit(&kv_empty[s]);
+            }
+            if (ok) {
+                umma_commit(&o_full[0]);
+                if (two) umma_commit(&o_full[1]);
+            }
+        }
+    } else if (warp >= 4) {
+        // ================= softmax, one query tile per warpgroup
+        const int i = (warp >= 8) ? 1 : 0;
+        if (i == 0 || two) {
+            const int r = tid - 128 * (i + 1);  // row in tile == TMEM lane
+            const int h = hh[i];
+            const int q = mm[i] * kBM + r;
+            int lo, hi;
+            row_bounds(P, b, q, lo, hi);
+            const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+            const uint32_t tS = tmem + lane_base + i * 128;
+            const uint32_t tO = tmem + lane_base + 256 + i * 128;
+            float m_used = -INFINITY, l = 0.f;
+            bool ok = nkt > 0;
+            for (int jj = 0; ok && jj < nkt; ++jj) {
+                ok = mbar_wait(&s_full[i], jj & 1, abort_flag, P.status);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const int k0 = (kt_begin + jj) * kBN;
+                uint32_t raw[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, reinterpret_cast<uint32_t(&)[32]>(raw[32 * c]));
+                tmem_ld_wait();
+                tmem_ld_fence(raw);
+                const bool full = (k0 >= lo) && (k0 + kBN - 1 <= hi);
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const float v = __uint_as_float(raw[c]);
+                    float x = (P.softcap > 0.f) ? capped_log2(v, P) : v * P.scale_log2;
+                    if (!full) {
+                        const int key = k0 + c;
+                        if (key < lo || key > hi) x = -INFINITY;
+                    }
+                    raw[c] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+                // rescale only when the running max grows by more than 2^8 (exact either way:
+                // O and l always share the same reference max)
+                const float m_new = fmaxf(m_used, mx);
+                const bool need = m_new > m_used + 8.0f;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = ex2(m_used - m_new);  // 0 when m_used = -inf
+                    m_used = m_new;
+                }
+                const float base = (m_used == -INFINITY) ? 0.f : m_used;
+                float rs = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2(__uint_as_float(raw[32 * c + 2 * e]) - base);
+                        const float p1 = ex2(__uint_as_float(raw[32 * c + 2 * e + 1]) - base);
+                        rs += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(tS + 16 * c, pk);
+                }
+                l = l * alpha + rs;
+                if (jj > 0 && __any_sync(0xffffffffu, need)) {
+                    // the previous PV has completed (it was issued before this S MMA)
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(tO + 32 * c, ov);
+                        tmem_ld_wait();
+                        tmem_ld_fence(ov);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st32(tO + 32 * c, ov);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&p_full[i]);
+            }
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[i], 0, abort_flag, P.status));
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+                const bool row_ok = q < P.T;
+                __nv_bfloat16* orow = A.o + (((size_t)b * P.T + (row_ok ? q : 0)) * P.Hq + h) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + 32 * c, ov);
+                    tmem_ld_wait();
+                    tmem_ld_fence(ov);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+                    if (row_ok) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
+                }
+                if (row_ok)
+                    A.lse[((size_t)b * P.Hq + h) * P.T + q] =
+                        (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                void* o, float* lse, cudaStream_t st) {
+    using C = FwdCfg<D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    FwdArgs A;
+    A.P = P;
+    A.o = static_cast<__nv_bfloat16*>(o);
+    A.lse = lse;
+    A.nqt = (P.T + kBM - 1) / kBM;
+    int items;
+    if (P.G >= 2) {
+        A.pairs = (P.G + 1) / 2;
+        items = P.B * P.Hkv * A.pairs * A.nqt;
+    } else {
+        A.pairs = (A.nqt + 1) / 2;
+        items = P.B * P.Hq * A.pairs;
+    }
+    k_attn_fwd<D><<<items, 384, C::SMEM, st>>>(tq, tk, tv, A);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                       float* lse, cudaStream_t st) {
+    switch (P.D) {
+        case 32: return launch_fwd_d<32>(P, tq, tk, tv, o, lse, st);
+        case 64: return launch_fwd_d<64>(P, tq, tk, tv, o, lse, st);
+        case 96: return launch_fwd_d<96>(P, tq, tk, tv, o, lse, st);
+        case 128: return launch_fwd_d<128>(P, tq, tk, tv, o, lse, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+int fwd_swizzle_bytes(int D) { return (D % 64 == 0) ? 128 : 64; }
+
+}  // namespace csa

@@ -1,0 +1,34 @@
+// csa_internal.h -- definitions shared by the host code and the kernels of libcsa.
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+// A bounded wait inside a kernel gives up after this many SM clocks (about a second).
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+constexpr int kBM = 128;  // query rows per tile (the MMA M)
+constexpr int kBN = 128;  // keys per tile
+
+// Everything a kernel needs to know about the problem.
+struct Problem {
+    int B, T, Hq, Hkv, D, G;
+    int causal, window;
+    float softcap;          // 0 = off
+    float scale;            // effective score scale
+    float scale_log2;       // scale * log2(e)
+    int rope, qk_norm;
+    float eps;
+    const int32_t* seg_start;  // [B, T] first index of each token's segment, or null
+    const int32_t* seg_end;    // [B, T] one past its last index, or null
+    const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
+    int* status;               // device status word (workspace)
+};
+
+// Kernel ids for the timing interface (order = csa_kernel_name()).
+enum KernelId { kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kDqFinalize, kNumKernels };
+
+}  // namespace csa

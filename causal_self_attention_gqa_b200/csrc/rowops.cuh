@@ -1,0 +1,47 @@
+// rowops.cuh -- small per-row helpers shared by the row kernels and the attention
+// kernels' epilogues: bf16 vector loads/stores, 16-lane group sums, transposed RoPE.
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace csa {
+
+__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* p, float (&f)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    f[0] = __low2float(a); f[1] = __high2float(a);
+    f[2] = __low2float(b); f[3] = __high2float(b);
+}
+__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        f[2 * i] = __low2float(h);
+        f[2 * i + 1] = __high2float(h);
+    }
+}
+__device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, const float (&f)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&a);
+    u.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+__device__ __forceinline__ float group16_sum(float v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, 16);
+    return v;
+}
+// Transpose of the rotate-half rotation by phi (i.e. rotation by -phi) applied to a
+// gradient pair (g_a at d, g_b at d + D/2); cs = (cos phi, sin phi).
+__device__ __forceinline__ void rope_transpose(float& ga, float& gb, float2 cs) {
+    const float a = ga, b = gb;
+    ga = a * cs.x + b * cs.y;
+    gb = b * cs.x - a * cs.y;
+}
+
+}  // namespace csa

@@ -1,0 +1,125 @@
+/*
+ * csa.h -- C ABI of libcsa.so: causal (or bidirectional) multi-head / grouped-query
+ * self-attention, forward and backward, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (per batch row b and query head h, with key/value head kv = h / (Hq/Hkv)):
+ *
+ *   q' = RoPE(RMSNorm(q)), k' = RoPE(RMSNorm(k))           (each step optional)
+ *   s_ij = scale * q'_i . k'_j,  s'_ij = c * tanh(s_ij / c)   (cap optional)
+ *   P_i  = softmax over the keys j visible to query i,  O_i = sum_j P_ij v_j
+ *   LSE_i = log sum_j exp(s'_ij)   (natural log, over the visible keys)
+ *
+ * Sources: the scaled dot-product attention equation and the causal (upper-triangular -inf)
+ * mask are those of the GPT-pretraining page (dekermanjian.github.io, llm_gpt_pretrain),
+ * section "Multihead Attention"; grouped-query heads, RoPE, QK-norm (parameter-free
+ * RMSNorm), logits soft-capping and RoPE from packed segment positions come from the
+ * nanogpt-jax-181m model card, section "Architecture", and packed rows with segment_ids
+ * from its section "SFT"; the sliding window from the flaxchat README, "Core Features".
+ * The pages give no formulas for RoPE, the norm, the cap or the window; the readings used
+ * here are stated at each field of csa_params.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are row-major and contiguous: q, o, dout, dq are [B, T, Hq, D] bf16;
+ *    k, v, dk, dv are [B, T, Hkv, D] bf16; lse is [B, Hq, T] fp32; segment_ids is [B, T] int32.
+ *    bf16 pointers are passed as void* and hold IEEE bfloat16 bit patterns.
+ *  - Every tensor pointer is a DEVICE pointer, allocated and owned by the caller, aligned to
+ *    16 bytes.  The workspace is caller-owned device memory of at least
+ *    csa_workspace_size() bytes, aligned to 256 bytes.  The library allocates no device
+ *    memory of its own in any call.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it and
+ *    the call returns without synchronising.  The only call that synchronises is
+ *    csa_device_status().
+ *  - Errors found on the host (bad shapes, pointers, workspace, device) are returned before
+ *    anything is enqueued; outputs are then untouched.  No call prints, aborts or throws.
+ *  - Errors found on the device (a bounded wait inside a kernel that ran out) are written
+ *    to a status word inside the workspace and read back with csa_device_status().
+ *  - Calls on the same workspace must not overlap on the device.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,     /* shape, head ratio, head dim, option value or NULL pointer   */
+    CSA_ERR_ALIGNMENT = 2,       /* a tensor pointer is not 16-byte (workspace: 256-byte) aligned */
+    CSA_ERR_WORKSPACE = 3,       /* workspace smaller than csa_workspace_size()                  */
+    CSA_ERR_ARCH = 4,            /* current device is not a compute-capability 10.0 GPU          */
+    CSA_ERR_LAUNCH = 5,          /* a kernel launch failed (cudaGetLastError after enqueue)      */
+    CSA_ERR_DEVICE_TIMEOUT = 6,  /* a bounded wait inside a kernel ran out (device-side)         */
+    CSA_ERR_CUDA = 7,            /* another CUDA runtime / driver call failed                    */
+    CSA_ERR_NOT_IMPLEMENTED = 8
+};
+
+/* Problem description.  B, T >= 0 (0 is an empty problem: nothing is enqueued, CSA_OK);
+ * Hq, Hkv >= 1 with Hq % Hkv == 0 (query head h uses key/value head h / (Hq / Hkv),
+ * contiguous groups); D in {32, 64, 96, 128}; T <= 1 << 20. */
+typedef struct csa_params {
+    int B, T, Hq, Hkv, D;
+    int causal;        /* 1: key j visible to query i only if j <= i (decoder self-attention);
+                          0: bidirectional                                                     */
+    int window;        /* <= 0: off; else causal: visible only if i - j < window (window keys
+                          including i); bidirectional: only if |i - j| < window              */
+    float softcap;     /* <= 0: off; else s' = softcap * tanh(s / softcap) on the scaled score,
+                          before the mask                                                      */
+    float rope_base;   /* <= 0: off; else rotate-half RoPE: for d < D/2, phi = pos * base^(-2d/D),
+                          (x_d, x_{d+D/2}) -> (x_d cos phi - x_{d+D/2} sin phi,
+                                               x_{d+D/2} cos phi + x_d sin phi);
+                          pos = index within the token's segment (= t without segment_ids)     */
+    int qk_norm;       /* 1: x -> x * (mean_d x^2 + qk_norm_eps)^(-1/2) on every q and k head
+                          vector, before RoPE; no learnable scale                              */
+    float qk_norm_eps; /* > 0 when qk_norm is on (1e-6 in the pages' models)                  */
+    float scale;       /* <= 0: 1 / sqrt(D); else the score scale                              */
+} csa_params;
+
+/* Bytes of workspace csa_attn_fwd (for_backward = 0) or csa_attn_bwd (for_backward = 1)
+ * needs for *p; 0 if *p is invalid.  A workspace sized for the backward also serves the
+ * forward. */
+size_t csa_workspace_size(const csa_params* p, int for_backward);
+
+/* Forward.  Reads the RAW q, k (before norm and RoPE) and v; writes o and lse.
+ * segment_ids may be NULL (one segment per row); otherwise tokens attend only within their
+ * maximal run of equal ids, and RoPE positions restart at 0 at each run's first token.
+ * Returns a status code (host-side checks); device-side problems: csa_device_status(). */
+int csa_attn_fwd(const csa_params* p, const void* q, const void* k, const void* v,
+                 const int32_t* segment_ids, void* o, float* lse, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* Backward.  Given the forward's inputs, its outputs o and lse, and dout = dL/do, writes
+ * dq, dk, dv = dL/d(raw q, k, v).  dk and dv of a key/value head sum the contributions of
+ * all query heads of its group.  Stateless: the norm / RoPE prologue is recomputed, so the
+ * workspace need not be the forward's. */
+int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o,
+                 const void* dout, const float* lse, const int32_t* segment_ids, void* dq, void* dk,
+                 void* dv, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
+ * last call that used it (CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA when the
+ * synchronisation itself failed).  Resets the recorded status to CSA_OK. */
+int csa_device_status(void* workspace, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* csa_status_string(int code);
+
+/* Kernel timing (for measurement).  While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the launch stream.  csa_timing_collect()
+ * synchronises those events, adds each kernel's elapsed times into `total_ms[k]` and its
+ * launch count into `launches[k]` for k < n (k indexes csa_kernel_name()), and forgets them.
+ * Not thread-safe. */
+int csa_timing_enable(int enable);
+int csa_timing_collect(double* total_ms, int* launches, int n);
+int csa_num_kernels(void);
+const char* csa_kernel_name(int k);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,159 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded bf16 inputs.
+
+Tolerances (stated for the bf16 path): O relative L2 <= 1e-2 and max-abs <= 2e-2;
+dQ, dK, dV relative L2 <= 2e-2 each; LSE max-abs <= 1e-2 (internal).
+Small shapes cover every option, ragged tails (T not a multiple of the 128-row tile),
+T = 1, odd group sizes and windows that bind.  The five named workloads run at full size
+in the launch configuration the benchmark times, checked against the oracle on sampled
+batch rows (batch rows are independent, so a row's outputs and gradients are exact
+oracle targets).
+"""
+import numpy as np
+import pytest
+import torch
+
+from causal_self_attention_gqa_b200.workloads import WORKLOADS, Workload, make_inputs, packed_segment_ids
+
+pytestmark = pytest.mark.gpu
+
+O_REL, O_ABS, G_REL, LSE_ABS = 1e-2, 2e-2, 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def csa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from causal_self_attention_gqa_b200 import _binding
+    return _binding
+
+
+@pytest.fixture(scope="module")
+def ora():
+    import oracle
+    oracle.build()
+    return oracle
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def run_gpu(csa, inp, opts, backward=True):
+    dev = torch.device("cuda:0")
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    seg = inp["segment_ids"].to(dev) if inp["segment_ids"] is not None else None
+    ws = csa.workspace_for(q, k, True, **opts)
+    o, lse = csa.attn_fwd(q, k, v, segment_ids=seg, workspace=ws, **opts)
+    out = dict(o=o, lse=lse)
+    if backward:
+        do = inp["do"].to(dev)
+        dq, dk, dv = csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, **opts)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert csa.device_status(ws) == 0
+    return {n: t.float().cpu().numpy() for n, t in out.items()}
+
+
+def check(gpu, ref_o, ref_lse, ref_g=None, rows=None):
+    sl = slice(None) if rows is None else rows
+    o = gpu["o"][sl]
+    assert np.all(np.isfinite(o))
+    r = rel_l2(o, ref_o)
+    m = float(np.max(np.abs(o - ref_o)))
+    assert r <= O_REL and m <= O_ABS, (r, m)
+    lse_err = float(np.max(np.abs(gpu["lse"][sl] - ref_lse)))
+    assert lse_err <= LSE_ABS, lse_err
+    if ref_g is not None:
+        for name, ref in zip(("dq", "dk", "dv"), ref_g):
+            g = gpu[name][sl]
+            assert np.all(np.isfinite(g)), name
+            e = rel_l2(g, ref)
+            assert e <= G_REL, (name, e)
+
+
+def _small(B, T, Hq, Hkv, D, seed, seg=None, **opts):
+    w = Workload("t", B=B, T=T, Hq=Hq, Hkv=Hkv, D=D, seed=seed, **opts)
+    inp = make_inputs(w)
+    if seg is not None:
+        inp["segment_ids"] = torch.from_numpy(packed_segment_ids(B, T, seg[0], seg[1], seed))
+    return w, inp
+
+
+SMALL = [
+    # (B, T, Hq, Hkv, D, options, segments)
+    (1, 1, 2, 1, 32, dict(), None),
+    (2, 17, 2, 2, 32, dict(), None),
+    (2, 128, 4, 2, 64, dict(), None),
+    (1, 129, 2, 1, 128, dict(), None),
+    (2, 300, 4, 2, 96, dict(), None),
+    (1, 300, 3, 1, 128, dict(), None),                      # odd group size (G = 3)
+    (2, 260, 2, 2, 32, dict(), None),                       # G = 1, odd number of query tiles
+    (1, 256, 4, 2, 128, dict(rope_base=10000.0), None),
+    (1, 256, 4, 2, 96, dict(qk_norm=True), None),
+    (2, 200, 4, 2, 64, dict(rope_base=10000.0, qk_norm=True), None),
+    (1, 300, 2, 1, 128, dict(rope_base=10000.0, qk_norm=True, softcap=50.0), None),
+    (1, 300, 2, 1, 64, dict(softcap=5.0), None),            # cap that binds (no norm)
+    (1, 520, 2, 1, 96, dict(window=100), None),             # window that binds, ragged
+    (2, 384, 4, 2, 128, dict(rope_base=10000.0, qk_norm=True, window=200), (20, 150)),
+    (1, 300, 2, 2, 32, dict(), (1, 40)),                    # segments, single-token documents
+    (1, 257, 4, 2, 64, dict(causal=False), None),
+    (1, 300, 2, 1, 128, dict(causal=False, window=64), None),
+    (2, 200, 2, 1, 96, dict(causal=False, rope_base=10000.0), (30, 90)),
+    (1, 200, 2, 2, 64, dict(scale=0.05), None),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}x{c[3]}D{c[4]}"
+                         + "".join(f"-{k}{v}" for k, v in c[5].items()) + ("-seg" if c[6] else ""))
+def test_small_shapes_match_oracle(csa, ora, case):
+    B, T, Hq, Hkv, D, opts, seg = case
+    w, inp = _small(B, T, Hq, Hkv, D, seed=7 + T + D, seg=seg, **opts)
+    kw = dict(w.options())
+    gpu = run_gpu(csa, inp, kw)
+    ref_o, ref_lse = ora.attn_fwd(inp["q"], inp["k"], inp["v"], segment_ids=inp["segment_ids"], **kw)
+    ref_g = ora.attn_bwd(inp["q"], inp["k"], inp["v"], inp["do"], segment_ids=inp["segment_ids"], **kw)
+    check(gpu, ref_o, ref_lse, ref_g)
+
+
+@pytest.mark.parametrize("widx", range(len(WORKLOADS)), ids=[w.name for w in WORKLOADS])
+def test_workload_full_size_sampled_rows(csa, ora, widx):
+    """Full-size run (the benchmark's launch configuration); oracle on sampled batch rows."""
+    w = WORKLOADS[widx]
+    inp = make_inputs(w)
+    kw = dict(w.options())
+    gpu = run_gpu(csa, inp, kw)
+    rows = [0] if w.B <= 2 else [0, w.B - 1]
+    if w.T <= 128:
+        rows = list(range(w.B))
+    for b in rows:
+        sl = slice(b, b + 1)
+        seg = inp["segment_ids"][sl] if inp["segment_ids"] is not None else None
+        args = (inp["q"][sl], inp["k"][sl], inp["v"][sl])
+        ref_o, ref_lse = ora.attn_fwd(*args, segment_ids=seg, **kw)
+        ref_g = ora.attn_bwd(*args, inp["do"][sl], segment_ids=seg, **kw)
+        check(gpu, ref_o, ref_lse, ref_g, rows=sl)
+
+
+def test_causal_outputs_ignore_future_tokens(csa):
+    """Masking is exact: changing tokens after position c leaves rows <= c bit-identical."""
+    w = Workload("t", B=1, T=384, Hq=4, Hkv=2, D=128, rope_base=10000.0, qk_norm=True, seed=3)
+    inp = make_inputs(w)
+    kw = w.options()
+    a = run_gpu(csa, inp, kw, backward=False)
+    cut = 200
+    inp2 = {k: (v.clone() if v is not None else None) for k, v in inp.items()}
+    for n in ("q", "k", "v"):
+        inp2[n][:, cut:] = -inp2[n][:, cut:]
+    b = run_gpu(csa, inp2, kw, backward=False)
+    assert np.array_equal(a["o"][:, :cut], b["o"][:, :cut])
+    assert np.array_equal(a["lse"][:, :, :cut], b["lse"][:, :, :cut])
+
+
+def test_repeated_calls_are_deterministic_in_forward(csa):
+    w = WORKLOADS[3].with_(B=2)
+    inp = make_inputs(w)
+    a = run_gpu(csa, inp, w.options(), backward=False)
+    b = run_gpu(csa, inp, w.options(), backward=False)
+    assert np.array_equal(a["o"], b["o"])
