@@ -15,7 +15,8 @@
 //   warp 0      TMA producer: K', V once; Q', dO tiles into a 2-stage ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 4-7   P / dS computation (thread = key row = TMEM lane), then the dK/dV epilogue
-//   warps 8-11  dQ' drain: TMEM -> fp32 reductions into the global accumulator
+//   warps 8-11  dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
+//               k_dq_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
 // written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
 // reuses the dP^T columns once dS has been formed.  dS^T goes to shared memory (128x128
@@ -454,9 +455,8 @@ __global__ void __launch_bounds__(384, 1)
                 if (q < P.T) {
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
-                        red_add_v4(dst + 32 * c + 4 * v4, __uint_as_float(v[4 * v4]) * P.scale,
-                                   __uint_as_float(v[4 * v4 + 1]) * P.scale, __uint_as_float(v[4 * v4 + 2]) * P.scale,
-                                   __uint_as_float(v[4 * v4 + 3]) * P.scale);
+                        red_add_v4(dst + 32 * c + 4 * v4, __uint_as_float(v[4 * v4]), __uint_as_float(v[4 * v4 + 1]),
+                                   __uint_as_float(v[4 * v4 + 2]), __uint_as_float(v[4 * v4 + 3]));
                 }
             }
             tc_fence_before();
