@@ -38,13 +38,14 @@ class Workload:
     rope_base: float = 0.0
     qk_norm: bool = False
     qk_norm_eps: float = 1e-6
+    scale: float = 0.0            # <= 0: 1/sqrt(D)
     seg_len: tuple | None = None  # (lo, hi) document lengths for packed rows
     seed: int = 0
 
     def options(self) -> dict:
         return dict(causal=self.causal, window=self.window, softcap=self.softcap,
                     rope_base=self.rope_base, qk_norm=self.qk_norm,
-                    qk_norm_eps=self.qk_norm_eps)
+                    qk_norm_eps=self.qk_norm_eps, scale=self.scale)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
