@@ -31,7 +31,7 @@ CSA_ERR_NOT_IMPLEMENTED = 8
 # every entry point include/csa.h declares
 EXPORTED = ["csa_workspace_size", "csa_attn_fwd", "csa_attn_bwd", "csa_device_status",
             "csa_status_string", "csa_timing_enable", "csa_timing_collect", "csa_num_kernels",
-            "csa_kernel_name"]
+            "csa_kernel_name", "csa_attn_fwd_static_scratch"]
 
 
 class Params(ctypes.Structure):
@@ -50,6 +50,8 @@ _lib.csa_attn_fwd.restype = ctypes.c_int
 _lib.csa_attn_bwd.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.c_size_t, _vp]
 _lib.csa_attn_bwd.restype = ctypes.c_int
+_lib.csa_attn_fwd_static_scratch.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.csa_attn_fwd_static_scratch.restype = ctypes.c_int
 _lib.csa_device_status.argtypes = [_vp, _vp]
 _lib.csa_device_status.restype = ctypes.c_int
 _lib.csa_status_string.argtypes = [ctypes.c_int]

@@ -376,3 +376,74 @@ const char* csa_kernel_name(int k) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ forward with library-owned scratch
+// For callers that cannot allocate device memory themselves (see csa_attn_fwd_static_scratch
+// in csa.h).  The scratch is one file-scope device array, loaded with the library and held
+// by every GPU that loads it until the process exits.
+namespace csa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)CSA_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device.  In host code the array's name
+// is only a host-side stand-in; the real address comes from cudaGetSymbolAddress, looked up
+// once per device (on the first call made with that device current) and cached.
+void* g_static_scratch_addr[64] = {nullptr};
+
+int static_scratch_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= 64) return CSA_ERR_CUDA;
+    if (!g_static_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return CSA_ERR_CUDA;
+        }
+        g_static_scratch_addr[dev] = p;
+    }
+    *out = g_static_scratch_addr[dev];
+    return CSA_OK;
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" int csa_attn_fwd_static_scratch(const csa_params* p, const void* q, const void* k, const void* v,
+                                           const int32_t* segment_ids, void* o, float* lse, int* device_status,
+                                           void* stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (p->B == 0 || p->T == 0) return CSA_OK;
+    if (!q || !k || !v || !o || !lse) return CSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        (segment_ids && !aligned(segment_ids, 4)) || (device_status && !aligned(device_status, 4)))
+        return CSA_ERR_ALIGNMENT;
+    // the problem's scratch must fit in the fixed array; nothing is allocated to make room
+    if (layout(*p, false, segment_ids != nullptr).total > kStaticScratchBytes) return CSA_ERR_WORKSPACE;
+    if ((rc = check_device())) return rc;
+    void* scratch = nullptr;
+    if ((rc = static_scratch_address(&scratch))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the status word is the only part that must start at zero: cleared by prepare();
+    // everything else the kernels read is rewritten by this call before it is read
+    Prepared pr;
+    if ((rc = prepare(p, false, q, k, segment_ids, scratch, kStaticScratchBytes, st, pr))) return rc;
+    if (device_status) {
+        if (cudaMemsetAsync(device_status, 0, sizeof(int), st) != cudaSuccess) {
+            cudaGetLastError();
+            return CSA_ERR_CUDA;
+        }
+        pr.P.status = device_status;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D))
+        return CSA_ERR_CUDA;
+    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, o, lse, st); });
+}

@@ -108,6 +108,37 @@ int csa_device_status(void* workspace, void* stream);
 /* Static, NUL-terminated description of a status code. */
 const char* csa_status_string(int code);
 
+/* Size of the library-owned scratch array used by csa_attn_fwd_static_scratch (16 MiB). */
+#define CSA_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Forward without a workspace argument, for callers that cannot allocate device memory:
+ * code that runs inside a host framework which owns every device allocation through its
+ * own allocator (and gives this caller none), or a latency-critical loop where a
+ * cudaMalloc, which may synchronise the device, is not acceptable.  The pages describe no
+ * such entry point; it has no counterpart there.
+ *
+ * Same arguments and results as csa_attn_fwd, minus the workspace.  Its scratch (status
+ * word, segment bounds, RoPE table, normalised q/k copies) lives in one file-scope device
+ * array of CSA_STATIC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine.
+ *  - A problem whose scratch would exceed CSA_STATIC_SCRATCH_BYTES (roughly
+ *    B*T*(Hq+Hkv)*D*2 bytes with QK-norm or RoPE, plus 8*B*T with segment_ids and 4*T*D with
+ *    RoPE) is rejected with CSA_ERR_WORKSPACE before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current and caches it; make that first call before any stream
+ *    capture.
+ *  - Every call shares the one array, which keeps the last call's contents.  The call
+ *    clears the status word it needs at zero and rewrites everything else before reading
+ *    it.  Calls that overlap on the GPU (different streams, or threads) race on the array
+ *    and give wrong results: serialise them.
+ *  - device_status: optional device pointer to one int; when non-NULL it is cleared and
+ *    receives the device-side status (CSA_ERR_DEVICE_TIMEOUT if a bounded wait ran out).
+ *    When NULL that status is only recorded inside the library's array. */
+int csa_attn_fwd_static_scratch(const csa_params* p, const void* q, const void* k, const void* v,
+                                const int32_t* segment_ids, void* o, float* lse, int* device_status,
+                                void* stream);
+
 /* Kernel timing (for measurement).  While enabled, every kernel the library launches is
  * bracketed by two CUDA events recorded on the launch stream.  csa_timing_collect()
  * synchronises those events, adds each kernel's elapsed times into `total_ms[k]` and its
