@@ -244,6 +244,24 @@ def config_dict(w, n):
             "l2": "flushed between timed steps (256 MiB write, outside the events)"}
 
 
+def profile_step(w):
+    """Warm-up step + one step of the path on cuda:0, for an ncu capture (-s/-c select it)."""
+    from causal_self_attention_gqa_b200 import _binding as csa
+    dev = torch.device("cuda:0")
+    inp = make_inputs(w)
+    kw = w.options()
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    seg = inp["segment_ids"].to(dev) if inp["segment_ids"] is not None else None
+    ws = csa.workspace_for(q, k, True, **kw)
+    for _ in range(2):
+        o, lse = csa.attn_fwd(q, k, v, segment_ids=seg, workspace=ws, **kw)
+        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    print(json.dumps({"profile_step": w.name, "B": w.B, "status": rc}))
+    return 0 if rc == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -253,8 +271,15 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end leg (default: min(K, 20))")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling cases)")
+    ap.add_argument("--profile-step", action="store_true",
+                    help="one warm-up step and one plain step, nothing else: a small case for ncu")
     args = ap.parse_args()
     w = BY_NAME[args.workload]
+    if args.batch > 0:
+        w = w.with_(B=args.batch)
+    if args.profile_step:
+        return profile_step(w)
     if args.impl == "reference":
         return run_reference(args, w)
 
