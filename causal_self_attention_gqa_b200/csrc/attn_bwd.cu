@@ -111,7 +111,7 @@ __device__ __forceinline__ void col_bounds(const Problem& P, int b, int j, int& 
     hi = h;
 }
 
-template <int D>
+template <int D, bool CAP>
 __global__ void __launch_bounds__(384, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -271,17 +271,24 @@ __global__ void __launch_bounds__(384, 1)
         uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
         const float kLog2e = 1.4426950408889634f;
         bool ok = nit > 0;
-        for (int it = 0; ok && it < nit; ++it) {
+        // this thread's LSE (log2 units) and delta for query row kr of iteration `it`, loaded
+        // from global one iteration ahead so the load latency hides behind the compute
+        auto fetch = [&](int it, float& l2, float& d) {
             const int h = kvh * P.G + it / nm;
+            const int q = (m_lo + it % nm) * kBM + kr;
+            const size_t o = ((size_t)b * P.Hq + h) * P.T + (q < P.T ? q : 0);
+            l2 = (q < P.T) ? A.lse[o] * kLog2e : INFINITY;
+            d = (q < P.T) ? A.delta[o] : 0.f;
+        };
+        float nl2 = INFINITY, nd = 0.f;
+        if (nit > 0) fetch(0, nl2, nd);
+        for (int it = 0; ok && it < nit; ++it) {
             const int m = m_lo + it % nm;
             const int q0 = m * kBM;
             const int buf = it & 1;
-            {
-                const int q = q0 + kr;
-                const size_t o = ((size_t)b * P.Hq + h) * P.T + q;
-                lse_s[buf * 128 + kr] = (q < P.T) ? A.lse[o] * kLog2e : INFINITY;
-                delta_s[buf * 128 + kr] = (q < P.T) ? A.delta[o] : 0.f;
-            }
+            lse_s[buf * 128 + kr] = nl2;
+            delta_s[buf * 128 + kr] = nd;
+            if (it + 1 < nit) fetch(it + 1, nl2, nd);
             mbar_arrive(wg_sync);
             ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
             ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status) &&
@@ -303,32 +310,36 @@ __global__ void __launch_bounds__(384, 1)
                 tmem_ld_fence(dpv);
                 uint32_t pk[16], dk16[16];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pp[2], dd[2];
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(ls + 32 * c + e);
+                    const float4 d4 = *reinterpret_cast<const float4*>(dl + 32 * c + e);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pp[4], dd[4];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int qi = 32 * c + e + u;
+                    for (int u = 0; u < 4; ++u) {
                         const float raw = __uint_as_float(sv[e + u]);
-                        float x, dfac = 1.f;
-                        if (P.softcap > 0.f) {
+                        float p, dfac = 1.f;
+                        if constexpr (CAP) {
                             const float y = raw * P.scale / P.softcap;
                             const float ex = ex2(y * 2.8853900817779268f);
                             const float t = 1.0f - __fdividef(2.0f, ex + 1.0f);
-                            x = P.softcap * kLog2e * t;
+                            p = ex2(fmaf(P.softcap * kLog2e, t, -lv[u]));
                             dfac = 1.0f - t * t;
                         } else {
-                            x = raw * P.scale_log2;
+                            p = ex2(fmaf(raw, P.scale_log2, -lv[u]));
                         }
-                        float p = ex2(x - ls[qi]);
                         if (!full) {
-                            const int q = q0 + qi;
+                            const int q = q0 + 32 * c + e + u;
                             if (q < lo || q > hi) p = 0.f;
                         }
                         pp[u] = p;
-                        dd[u] = p * (__uint_as_float(dpv[e + u]) - dl[qi]) * dfac;
+                        dd[u] = p * (__uint_as_float(dpv[e + u]) - dv4[u]) * dfac;
                     }
                     pk[e / 2] = pack_bf16x2(pp[0], pp[1]);
+                    pk[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
                     dk16[e / 2] = pack_bf16x2(dd[0], dd[1]);
+                    dk16[e / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
                 }
                 tmem_st16(t_s + 16 * c, pk);  // P^T (bf16) over S^T columns already read
                 // dS^T row kr, queries [32c, 32c+32): 4 chunks of 16 bytes, 128-byte swizzle
@@ -472,14 +483,15 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int D>
-static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+template <int D, bool CAP>
+static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc,
                                 const void* k_raw, void* dk, void* dv, cudaStream_t st) {
     using C = BwdCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e =
+            cudaFuncSetAttribute(k_attn_bwd<D, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -493,8 +505,16 @@ static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const C
     A.dv = static_cast<__nv_bfloat16*>(dv);
     A.nkt = (P.T + kBN - 1) / kBN;
     const int grid = A.nkt * P.B * P.Hkv;
-    k_attn_bwd<D><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, A);
+    k_attn_bwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, A);
     return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc,
+                                const void* k_raw, void* dk, void* dv, cudaStream_t st) {
+    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st)
+                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
 }
 
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

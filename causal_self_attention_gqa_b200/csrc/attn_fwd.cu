@@ -105,7 +105,7 @@ __device__ __forceinline__ float capped_log2(float raw, const Problem& P) {
     return P.softcap * 1.4426950408889634f * t;
 }
 
-template <int D>
+template <int D, bool CAP>
 __global__ void __launch_bounds__(384, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdArgs A) {
@@ -300,19 +300,26 @@ __global__ void __launch_bounds__(384, 1)
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, reinterpret_cast<uint32_t(&)[32]>(raw[32 * c]));
                 tmem_ld_wait();
                 tmem_ld_fence(raw);
-                const bool full = (k0 >= lo) && (k0 + kBN - 1 <= hi);
-                float mx = -INFINITY;
+                // logits in log2 units: with the cap x = c log2(e) tanh(s / c) (computed here);
+                // without it x = raw * scale_log2, so the max and the mask work on the raw
+                // scores and the scale folds into the exponent's FFMA (scale > 0)
+                if constexpr (CAP) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const float v = __uint_as_float(raw[c]);
-                    float x = (P.softcap > 0.f) ? capped_log2(v, P) : v * P.scale_log2;
-                    if (!full) {
-                        const int key = k0 + c;
-                        if (key < lo || key > hi) x = -INFINITY;
-                    }
-                    raw[c] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                    for (int c = 0; c < 128; ++c) raw[c] = __float_as_uint(capped_log2(__uint_as_float(raw[c]), P));
                 }
+                const bool full = (k0 >= lo) && (k0 + kBN - 1 <= hi);
+                if (!full) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) {
+                        const int key = k0 + c;
+                        if (key < lo || key > hi) raw[c] = 0xff800000u;  // -inf
+                    }
+                }
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(raw[c]));
+                const float xmul = CAP ? 1.0f : P.scale_log2;
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * xmul;
                 // rescale only when the running max grows by more than 2^8 (exact either way:
                 // O and l always share the same reference max)
                 const float m_new = fmaxf(m_used, mx);
@@ -322,20 +329,21 @@ __global__ void __launch_bounds__(384, 1)
                     alpha = ex2(m_used - m_new);  // 0 when m_used = -inf
                     m_used = m_new;
                 }
-                const float base = (m_used == -INFINITY) ? 0.f : m_used;
-                float rs = 0.f;
+                const float nbase = (m_used == -INFINITY) ? 0.f : -m_used;
+                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(__uint_as_float(raw[32 * c + 2 * e]) - base);
-                        const float p1 = ex2(__uint_as_float(raw[32 * c + 2 * e + 1]) - base);
-                        rs += p0 + p1;
+                        const float p0 = ex2(fmaf(__uint_as_float(raw[32 * c + 2 * e]), xmul, nbase));
+                        const float p1 = ex2(fmaf(__uint_as_float(raw[32 * c + 2 * e + 1]), xmul, nbase));
+                        rs4[e & 3] += p0 + p1;
                         pk[e] = pack_bf16x2(p0, p1);
                     }
                     tmem_st16(tS + 16 * c, pk);
                 }
+                const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
                 l = l * alpha + rs;
                 if (jj > 0 && __any_sync(0xffffffffu, need)) {
                     // the previous PV has completed (it was issued before this S MMA)
@@ -392,13 +400,14 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int D>
-static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+template <int D, bool CAP>
+static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 void* o, float* lse, cudaStream_t st) {
     using C = FwdCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e =
+            cudaFuncSetAttribute(k_attn_fwd<D, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -415,8 +424,15 @@ static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const C
         A.pairs = (A.nqt + 1) / 2;
         items = P.B * P.Hq * A.pairs;
     }
-    k_attn_fwd<D><<<items, 384, C::SMEM, st>>>(tq, tk, tv, A);
+    k_attn_fwd<D, CAP><<<items, 384, C::SMEM, st>>>(tq, tk, tv, A);
     return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                void* o, float* lse, cudaStream_t st) {
+    return (P.softcap > 0.f) ? launch_fwd_cap<D, true>(P, tq, tk, tv, o, lse, st)
+                             : launch_fwd_cap<D, false>(P, tq, tk, tv, o, lse, st);
 }
 
 cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
