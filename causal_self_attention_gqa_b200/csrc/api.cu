@@ -20,7 +20,7 @@ cudaError_t launch_dq_finalize(const Problem& P, const float* dq_acc, const void
 cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                        float* lse, cudaStream_t st);
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
                        void* dk, void* dv, cudaStream_t st);
 
 namespace {
@@ -135,6 +135,21 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
                           sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// [B, T, H, D] fp32 accumulator for TMA reduce-adds: boxes of 16 floats x 1 head x 128 rows x
+// 1 batch, 64-byte swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)T * H * D * 4};
+    cuuint32_t box[4] = {16, 1, (cuuint32_t)kBM, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -300,12 +315,13 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
     float* delta = reinterpret_cast<float*>(w + pr.L.delta);
     float* dq_acc = reinterpret_cast<float*>(w + pr.L.dq_acc);
     if ((rc = timed(kBwdPre, st, [&] { return launch_bwd_pre(pr.P, o, dout, delta, dq_acc, st); }))) return rc;
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
-        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&tdo, dout, p->B, p->T, p->Hq, p->D))
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&tdo, dout, p->B, p->T, p->Hq, p->D) ||
+        !make_map_f32(&tdq, dq_acc, p->B, p->T, p->Hq, p->D))
         return CSA_ERR_CUDA;
     if ((rc = timed(kBwd, st,
-                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, lse, delta, dq_acc, k, dk, dv, st); })))
+                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k, dk, dv, st); })))
         return rc;
     return timed(kDqFinalize, st, [&] { return launch_dq_finalize(pr.P, dq_acc, q, dq, st); });
 }

@@ -50,8 +50,8 @@ struct BwdCfg {
     static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
     static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
     // kv_full, q_full[2], do_full[2], stage_empty[2], s_full, dp_full, ds_full, ds_free,
-    // dq_full, dq_empty, acc_full, wg_sync
-    static constexpr int NBAR = 15;
+    // dq_full, dq_empty, acc_full, wg_sync, drain_sync
+    static constexpr int NBAR = 16;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -115,7 +115,7 @@ template <int D, bool CAP>
 __global__ void __launch_bounds__(384, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const BwdArgs A) {
+               const __grid_constant__ CUtensorMap tm_dq, const BwdArgs A) {
     using C = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const Problem& P = A.P;
@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* dq_full = bars + 11;
     uint64_t* dq_empty = bars + 12;
     uint64_t* acc_full = bars + 13;
-    uint64_t* wg_sync = bars + 14;  // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
+    uint64_t* wg_sync = bars + 14;     // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
+    uint64_t* drain_sync = bars + 15;  // the dQ drain warpgroup's own barrier
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&do_full[s], 1);
-            mbar_init(&stage_empty[s], 1);
+            mbar_init(&stage_empty[s], 2);  // MMA commit + drain (staging read by the reduce)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(dq_empty, 128);
         mbar_init(acc_full, 1);
         mbar_init(wg_sync, 128);
+        mbar_init(drain_sync, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -446,33 +448,60 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp >= 8) {
         // ================= dQ' drain (thread = query row of the current tile)
+        // TMEM -> registers -> fp32 tile in shared memory -> TMA reduce-add into the global
+        // accumulator.  The staging space is the finished stage's Q' and dO tiles (their MMAs
+        // are complete once dQ' is): together they hold exactly the 128 x D fp32 tile, as
+        // D/16 boxes of 16 floats x 128 rows in the 64-byte swizzle.  The dQ' columns are
+        // released as soon as they are read; the stage is released to the producer once the
+        // reduce has read the staging.
         const int r = tid - 256;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_dq = tmem + lane_base + 384;
+        constexpr int kAtoms = D / 16;  // 8 KB each
         bool ok = nit > 0;
         for (int it = 0; ok && it < nit; ++it) {
+            const int s = it & 1;
             const int h = kvh * P.G + it / nm;
-            const int q = (m_lo + it % nm) * kBM + r;
+            const int q0 = (m_lo + it % nm) * kBM;
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
             if (!ok) break;
             tc_fence_after();
-            float* dst = A.dq_acc + (((size_t)b * P.T + (q < P.T ? q : 0)) * P.Hq + h) * D;
+            auto atom_base = [&](int a) -> uint8_t* {
+                return (a < kAtoms / 2) ? smem + C::OFF_Q + s * C::TILE + a * 8192
+                                        : smem + C::OFF_DO + s * C::TILE + (a - kAtoms / 2) * 8192;
+            };
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(t_dq + 32 * c, v);
                 tmem_ld_wait();
                 tmem_ld_fence(v);
-                if (q < P.T) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        red_add_v4(dst + 32 * c + 4 * v4, __uint_as_float(v[4 * v4]), __uint_as_float(v[4 * v4 + 1]),
-                                   __uint_as_float(v[4 * v4 + 2]), __uint_as_float(v[4 * v4 + 3]));
+                for (int half = 0; half < 2; ++half) {
+                    uint8_t* row = atom_base(2 * c + half) + r * 64;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int pc = j ^ ((r >> 1) & 3);
+                        *reinterpret_cast<uint4*>(row + pc * 16) =
+                            make_uint4(v[16 * half + 4 * j], v[16 * half + 4 * j + 1], v[16 * half + 4 * j + 2],
+                                       v[16 * half + 4 * j + 3]);
+                    }
                 }
             }
             tc_fence_before();
-            mbar_arrive(dq_empty);
+            mbar_arrive(dq_empty);  // the dQ' columns may be overwritten now
+            fence_proxy_async_smem();
+            mbar_arrive(drain_sync);
+            ok = __all_sync(0xffffffffu, mbar_wait(drain_sync, it & 1, abort_flag, P.status));
+            if (!ok) break;
+            if (r == 0) {
+                for (int a = 0; a < kAtoms; ++a) tma_reduce_add_4d(&tm_dq, atom_base(a), a * 16, h, q0, b);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(&stage_empty[s]);  // second arrival: staging read, stage reusable
+            }
         }
+        if (r == 0) bulk_wait_group0();
     }
 
     tc_fence_before();
@@ -485,7 +514,7 @@ __global__ void __launch_bounds__(384, 1)
 
 template <int D, bool CAP>
 static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc,
+                                const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
                                 const void* k_raw, void* dk, void* dv, cudaStream_t st) {
     using C = BwdCfg<D>;
     static bool attr_set = false;
@@ -505,26 +534,26 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.dv = static_cast<__nv_bfloat16*>(dv);
     A.nkt = (P.T + kBN - 1) / kBN;
     const int grid = A.nkt * P.B * P.Hkv;
-    k_attn_bwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, A);
+    k_attn_bwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, A);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc,
+                                const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
                                 const void* k_raw, void* dk, void* dv, cudaStream_t st) {
-    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st)
-                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st)
+                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
 }
 
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
                        void* dk, void* dv, cudaStream_t st) {
     switch (P.D) {
-        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
         default: return cudaErrorInvalidValue;
     }
 }
