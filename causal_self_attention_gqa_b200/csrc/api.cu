@@ -16,12 +16,13 @@ cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start
 cudaError_t launch_prologue(const Problem& P, const void* q, const void* k, void* qo, void* ko, cudaStream_t st);
 cudaError_t launch_bwd_pre(const Problem& P, const void* o, const void* dout, float* delta, float* dq_acc,
                            cudaStream_t st);
-cudaError_t launch_dq_finalize(const Problem& P, const float* dq_acc, const void* q, void* dq, cudaStream_t st);
+cudaError_t launch_grad_finalize(const Problem& P, const float* dq_acc, const float* dk_acc, const void* q,
+                                 const void* k, void* dq, void* dk, cudaStream_t st);
 cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                        float* lse, cudaStream_t st);
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
-                       void* dk, void* dv, cudaStream_t st);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
+                       float* dk_acc, void* dk, void* dv, cudaStream_t st);
 
 namespace {
 
@@ -30,7 +31,8 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-    size_t status = 0, seg_start = 0, seg_end = 0, rope = 0, qp = 0, kp = 0, delta = 0, dq_acc = 0, total = 0;
+    size_t status = 0, seg_start = 0, seg_end = 0, rope = 0, qp = 0, kp = 0, delta = 0, dq_acc = 0, dk_acc = 0,
+           total = 0;
 };
 
 bool needs_prologue(const csa_params& p) { return p.qk_norm != 0 || p.rope_base > 0.f; }
@@ -62,6 +64,10 @@ Layout layout(const csa_params& p, bool backward, bool has_seg) {
         off += up(BT * p.Hq * 4);
         L.dq_acc = off;
         off += up(BT * p.Hq * p.D * 4);
+        if (needs_prologue(p)) {
+            L.dk_acc = off;
+            off += up(BT * p.Hkv * p.D * 4);
+        }
     }
     L.total = off;
     return L;
@@ -314,6 +320,7 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
     uint8_t* w = static_cast<uint8_t*>(workspace);
     float* delta = reinterpret_cast<float*>(w + pr.L.delta);
     float* dq_acc = reinterpret_cast<float*>(w + pr.L.dq_acc);
+    float* dk_acc = needs_prologue(*p) ? reinterpret_cast<float*>(w + pr.L.dk_acc) : nullptr;
     if ((rc = timed(kBwdPre, st, [&] { return launch_bwd_pre(pr.P, o, dout, delta, dq_acc, st); }))) return rc;
     CUtensorMap tq, tk, tv, tdo, tdq;
     if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
@@ -321,9 +328,10 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
         !make_map_f32(&tdq, dq_acc, p->B, p->T, p->Hq, p->D))
         return CSA_ERR_CUDA;
     if ((rc = timed(kBwd, st,
-                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k, dk, dv, st); })))
+                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st); })))
         return rc;
-    return timed(kDqFinalize, st, [&] { return launch_dq_finalize(pr.P, dq_acc, q, dq, st); });
+    return timed(kGradFinalize, st,
+                 [&] { return launch_grad_finalize(pr.P, dq_acc, dk_acc, q, k, dq, dk, st); });
 }
 
 int csa_device_status(void* workspace, void* stream) {
@@ -387,7 +395,7 @@ int csa_num_kernels(void) { return kNumKernels; }
 
 const char* csa_kernel_name(int k) {
     static const char* names[kNumKernels] = {"k_prep", "k_qk_prologue", "k_attn_fwd",
-                                             "k_bwd_pre", "k_attn_bwd", "k_dq_finalize"};
+                                             "k_bwd_pre", "k_attn_bwd", "k_grad_finalize"};
     return (k >= 0 && k < kNumKernels) ? names[k] : "";
 }
 

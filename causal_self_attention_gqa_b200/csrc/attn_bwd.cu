@@ -6,7 +6,7 @@
 //     dV_j  += sum_i P_ij dO_i
 //     dS_ij  = P_ij (dP_ij - delta_i) * (1 - tanh^2(s_ij / c))      (last factor: cap only)
 //     dQ'_i += scale sum_j dS_ij k'_j        dK'_j += scale sum_i dS_ij q'_i
-// followed by the transposed RoPE and RMSNorm on dK' (epilogue here) and dQ' (k_dq_finalize).
+// followed by the transposed RoPE and RMSNorm on dK' and dQ' (k_grad_finalize).
 //
 // One CTA owns a 128-key tile of one (b, kv head) and loops over the G query heads of the
 // group and every 128-row query tile that sees those keys, so dK and dV of the group sum in
@@ -14,12 +14,13 @@
 // Warp roles (384 threads):
 //   warp 0      TMA producer: K', V once; Q', dO tiles into a 2-stage ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 4-7   P / dS computation (thread = key row = TMEM lane), then the dK/dV epilogue
+//   warps 4-7   P / dS computation (thread = key row = TMEM lane), then the dK'/dV epilogue
 //   warps 8-11  dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
-//               k_dq_finalize applies the score scale)
+//               k_grad_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
 // written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
-// reuses the dP^T columns once dS has been formed.  dS^T goes to shared memory (128x128
+// then reuses the S^T columns.  MMA order per tile: dV, dK, dQ' of tile i, dP^T of tile
+// i+1 (no wait on the drain), then S^T of tile i+1 once the drain has read dQ'.  dS^T goes to shared memory (128x128
 // bf16, 128-byte swizzle) where it is the K-major A operand of dK' and, read MN-major,
 // the A operand of dQ'.
 #include <cuda.h>
@@ -65,7 +66,7 @@ struct BwdArgs {
     const float* lse;      // [B, Hq, T] natural log
     const float* delta;    // [B, Hq, T]
     float* dq_acc;         // [B, T, Hq, D] fp32, zeroed
-    const __nv_bfloat16* k_raw;  // raw K (for the RMSNorm backward of dK)
+    float* dk_acc;         // [B, T, Hkv, D] fp32 raw dK' (QK-norm or RoPE on), else unused
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     int nkt;  // key tiles per (b, kv head)
@@ -222,24 +223,31 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t sq = smem_u32(smem + C::OFF_Q), sdo = smem_u32(smem + C::OFF_DO);
             const uint32_t sds = smem_u32(smem + C::OFF_DS);
             const uint32_t t_dv = tmem, t_dk = tmem + 128, t_s = tmem + 256, t_dp = tmem + 384;
-            bool ok = mbar_wait(kv_full, 0, abort_flag, P.status);
-            for (int it = 0; ok && it < nit; ++it) {
-                const int s = it & 1, ph = (it >> 1) & 1;
-                if (!(ok = mbar_wait(&q_full[s], ph, abort_flag, P.status))) break;
-                tc_fence_after();
-                // S^T = K' Q'^T  (M = 128 keys, N = 128 queries, K = D)
+            // S^T = K' Q'^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D)
+            auto issue_s = [&](int st) {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_ss(t_s, bdesc_kmajor<D>(sk, ks), bdesc_kmajor<D>(sq + s * C::TILE, ks), C::IDESC_S, ks > 0);
+                    umma_ss(t_s, bdesc_kmajor<D>(sk, ks), bdesc_kmajor<D>(sq + st * C::TILE, ks), C::IDESC_S, ks > 0);
                 umma_commit(s_full);
-                if (!(ok = mbar_wait(&do_full[s], ph, abort_flag, P.status))) break;
-                if (it > 0 && !(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, P.status))) break;
-                tc_fence_after();
-                // dP^T = V dO^T
+            };
+            auto issue_dp = [&](int st) {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_ss(t_dp, bdesc_kmajor<D>(sv, ks), bdesc_kmajor<D>(sdo + s * C::TILE, ks), C::IDESC_S, ks > 0);
+                    umma_ss(t_dp, bdesc_kmajor<D>(sv, ks), bdesc_kmajor<D>(sdo + st * C::TILE, ks), C::IDESC_S, ks > 0);
                 umma_commit(dp_full);
+            };
+            bool ok = mbar_wait(kv_full, 0, abort_flag, P.status) && mbar_wait(&q_full[0], 0, abort_flag, P.status);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+                ok = mbar_wait(&do_full[0], 0, abort_flag, P.status);
+                if (ok) {
+                    tc_fence_after();
+                    issue_dp(0);
+                }
+            }
+            for (int it = 0; ok && it < nit; ++it) {
+                const int s = it & 1;
                 if (!(ok = mbar_wait(ds_full, it & 1, abort_flag, P.status))) break;
                 tc_fence_after();
                 // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
@@ -252,13 +260,27 @@ __global__ void __launch_bounds__(384, 1)
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ss(t_dk, ds_desc_kmajor(sds, ks), bdesc_mnmajor<D>(sq + s * C::TILE, ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
-                // dQ' = dS K'  (A = dS, MN-major view of the same tile; B = K', MN-major)
+                // dQ' = dS K' into the S^T columns (P^T there is consumed by the dV MMA issued
+                // above; MMAs of one thread run in issue order)
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
-                    umma_ss(t_dp, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
+                    umma_ss(t_s, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
                 umma_commit(dq_full);
                 umma_commit(&stage_empty[s]);
                 umma_commit(ds_free);
+                if (it + 1 < nit) {
+                    const int s1 = (it + 1) & 1, ph1 = ((it + 1) >> 1) & 1;
+                    // dP^T of the next tile right away: its columns were read before ds_full
+                    if (!(ok = mbar_wait(&do_full[s1], ph1, abort_flag, P.status))) break;
+                    tc_fence_after();
+                    issue_dp(s1);
+                    // S^T of the next tile once the drain has read dQ' out of those columns
+                    if (!(ok = mbar_wait(&q_full[s1], ph1, abort_flag, P.status) &&
+                               mbar_wait(dq_empty, it & 1, abort_flag, P.status)))
+                        break;
+                    tc_fence_after();
+                    issue_s(s1);
+                }
             }
             if (ok) umma_commit(acc_full);
         }
@@ -380,69 +402,33 @@ __global__ void __launch_bounds__(384, 1)
                                              pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7])));
                 }
             }
-            // dK = RMSNorm^T(RoPE^T(scale * dK')), two passes over 16-pair chunks (lo, hi halves)
+            // dK': with QK-norm or RoPE the raw fp32 sum goes to the workspace and the
+            // finalize kernel applies scale, RoPE^T and the RMSNorm backward (a bandwidth-bound
+            // pass); without them dK = scale * dK' is written here.
             const uint32_t t_dk = tmem + lane_base + 128;
-            constexpr int kHalf = D / 2;
-            const int pos = row_ok ? (P.seg_start ? key - P.seg_start[(size_t)b * P.T + key] : key) : 0;
-            const __nv_bfloat16* xr = A.k_raw + row_off;
-            float ss = 0.f, dot = 0.f;
-            if (P.qk_norm) {
+            const bool transform = P.rope || P.qk_norm;
 #pragma unroll 1
-                for (int c = 0; c < kHalf / 16; ++c) {
-                    uint32_t ulo[16], uhi[16];
-                    tmem_ld16(t_dk + 16 * c, ulo);
-                    tmem_ld16(t_dk + kHalf + 16 * c, uhi);
-                    tmem_ld_wait();
-                    tmem_ld_fence(ulo);
-                    tmem_ld_fence(uhi);
-#pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        float xl[4] = {0.f, 0.f, 0.f, 0.f}, xh[4] = {0.f, 0.f, 0.f, 0.f};
-                        if (row_ok) {
-                            load_bf16x4(xr + 16 * c + e, xl);
-                            load_bf16x4(xr + kHalf + 16 * c + e, xh);
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            float ga = __uint_as_float(ulo[e + u]) * P.scale;
-                            float gb = __uint_as_float(uhi[e + u]) * P.scale;
-                            if (P.rope) rope_transpose(ga, gb, P.rope_cs[(size_t)pos * kHalf + 16 * c + e + u]);
-                            ss += xl[u] * xl[u] + xh[u] * xh[u];
-                            dot += ga * xl[u] + gb * xh[u];
-                        }
-                    }
-                }
-            }
-            const float rs = P.qk_norm ? 1.0f / sqrtf(ss / (float)D + P.eps) : 1.f;
-            const float k3 = P.qk_norm ? rs * rs * rs * dot / (float)D : 0.f;
-#pragma unroll 1
-            for (int c = 0; c < kHalf / 16; ++c) {
-                uint32_t ulo[16], uhi[16];
-                tmem_ld16(t_dk + 16 * c, ulo);
-                tmem_ld16(t_dk + kHalf + 16 * c, uhi);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(t_dk + 32 * c, v);
                 tmem_ld_wait();
-                tmem_ld_fence(ulo);
-                tmem_ld_fence(uhi);
+                tmem_ld_fence(v);
+                if (!row_ok) continue;
+                if (transform) {
+                    uint4* dst = reinterpret_cast<uint4*>(A.dk_acc + row_off + 32 * c);
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    float xl[4] = {0.f, 0.f, 0.f, 0.f}, xh[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (row_ok && P.qk_norm) {
-                        load_bf16x4(xr + 16 * c + e, xl);
-                        load_bf16x4(xr + kHalf + 16 * c + e, xh);
-                    }
-                    float ol[4], oh[4];
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        dst[v4] = make_uint4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(A.dk + row_off + 32 * c);
+                    const float sc = P.scale;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float ga = __uint_as_float(ulo[e + u]) * P.scale;
-                        float gb = __uint_as_float(uhi[e + u]) * P.scale;
-                        if (P.rope) rope_transpose(ga, gb, P.rope_cs[(size_t)pos * kHalf + 16 * c + e + u]);
-                        ol[u] = rs * ga - k3 * xl[u];
-                        oh[u] = rs * gb - k3 * xh[u];
-                    }
-                    if (row_ok) {
-                        store_bf16x4(A.dk + row_off + 16 * c + e, ol);
-                        store_bf16x4(A.dk + row_off + kHalf + 16 * c + e, oh);
-                    }
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * v4]) * sc, __uint_as_float(v[8 * v4 + 1]) * sc),
+                            pack_bf16x2(__uint_as_float(v[8 * v4 + 2]) * sc, __uint_as_float(v[8 * v4 + 3]) * sc),
+                            pack_bf16x2(__uint_as_float(v[8 * v4 + 4]) * sc, __uint_as_float(v[8 * v4 + 5]) * sc),
+                            pack_bf16x2(__uint_as_float(v[8 * v4 + 6]) * sc, __uint_as_float(v[8 * v4 + 7]) * sc));
                 }
             }
         }
@@ -456,8 +442,8 @@ __global__ void __launch_bounds__(384, 1)
         // reduce has read the staging.
         const int r = tid - 256;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_dq = tmem + lane_base + 384;
-        constexpr int kAtoms = D / 16;  // 8 KB each
+        const uint32_t t_dq = tmem + lane_base + 256;  // dQ' shares the S^T columns
+        constexpr int kAtoms = D / 16;                   // 8 KB each
         bool ok = nit > 0;
         for (int it = 0; ok && it < nit; ++it) {
             const int s = it & 1;
@@ -515,7 +501,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int D, bool CAP>
 static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
-                                const void* k_raw, void* dk, void* dv, cudaStream_t st) {
+                                float* dk_acc, void* dk, void* dv, cudaStream_t st) {
     using C = BwdCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -529,7 +515,7 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.lse = lse;
     A.delta = delta;
     A.dq_acc = dq_acc;
-    A.k_raw = static_cast<const __nv_bfloat16*>(k_raw);
+    A.dk_acc = dk_acc;
     A.dk = static_cast<__nv_bfloat16*>(dk);
     A.dv = static_cast<__nv_bfloat16*>(dv);
     A.nkt = (P.T + kBN - 1) / kBN;
@@ -541,19 +527,19 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
 template <int D>
 static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
-                                const void* k_raw, void* dk, void* dv, cudaStream_t st) {
-    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st)
-                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
+                                float* dk_acc, void* dk, void* dv, cudaStream_t st) {
+    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st)
+                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
 }
 
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, const void* k_raw,
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, float* dk_acc,
                        void* dk, void* dv, cudaStream_t st) {
     switch (P.D) {
-        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
-        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, k_raw, dk, dv, st);
+        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
+        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
+        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
+        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -29,6 +29,6 @@ struct Problem {
 };
 
 // Kernel ids for the timing interface (order = csa_kernel_name()).
-enum KernelId { kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kDqFinalize, kNumKernels };
+enum KernelId { kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kNumKernels };
 
 }  // namespace csa

@@ -3,7 +3,8 @@
 //                  RoPE (cos, sin) table for positions 0..T-1, computed in fp64
 //   k_qk_prologue  q' = RoPE(RMSNorm(q)), k' = RoPE(RMSNorm(k)) -> bf16 copies in the workspace
 //   k_bwd_pre      delta_i = sum_d dO_id O_id per (b, h, i) and a zeroed fp32 dQ accumulator
-//   k_dq_finalize  dq = RMSNorm^T(RoPE^T(scale * dQ accumulator)) -> bf16
+//   k_grad_finalize dq (and dk when QK-norm or RoPE is on) = RMSNorm^T(RoPE^T(scale * acc))
+//                  -> bf16, from the fp32 dQ' accumulator and the raw dK' sums
 //
 // The norm is the parameter-free RMSNorm and the rotation the rotate-half RoPE of the
 // nanogpt-jax-181m model card ("Architecture"); positions restart at each packed segment
@@ -177,36 +178,48 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const __nv_bfloat16* __restrict
     }
 }
 
-// ------------------------------------------------------------------ dQ finalize
+// ------------------------------------------------------------------ gradient finalize
+// Rows [0, rows_q): dq = RMSNorm^T(RoPE^T(scale * dQ')) from the fp32 accumulator and raw q.
+// Rows [rows_q, rows_q + rows_k): the same for dk from raw dK' and raw k (only when QK-norm
+// or RoPE is on; otherwise the attention kernel already wrote dk).
 template <int D>
-__global__ void __launch_bounds__(256) k_dq_finalize(const float* __restrict__ dq_acc,
-                                                     const __nv_bfloat16* __restrict__ q,
-                                                     __nv_bfloat16* __restrict__ dq, Problem P, long long rows) {
+__global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__ dq_acc,
+                                                       const float* __restrict__ dk_acc,
+                                                       const __nv_bfloat16* __restrict__ q,
+                                                       const __nv_bfloat16* __restrict__ k,
+                                                       __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                                                       Problem P, long long rows_q, long long rows_total) {
     constexpr int kHalf = D / 2;
     const int lane16 = threadIdx.x & 15;
     const long long row_raw = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
-    const bool valid = row_raw < rows;  // no early return: the group shuffles need every lane
-    const long long row = valid ? row_raw : 0;
+    const bool valid = row_raw < rows_total;  // no early return: the group shuffles need every lane
+    const long long row0 = valid ? row_raw : 0;
+    const bool is_q = row0 < rows_q;
+    const long long row = is_q ? row0 : row0 - rows_q;
+    const int H = is_q ? P.Hq : P.Hkv;
+    const float* acc = is_q ? dq_acc : dk_acc;
+    const __nv_bfloat16* x = is_q ? q : k;
+    __nv_bfloat16* out = is_q ? dq : dk;
     const bool active = valid && lane16 < D / 8;
     const int d0 = 4 * lane16;
     float u_lo[4] = {0.f, 0.f, 0.f, 0.f}, u_hi[4] = {0.f, 0.f, 0.f, 0.f};
     float x_lo[4] = {0.f, 0.f, 0.f, 0.f}, x_hi[4] = {0.f, 0.f, 0.f, 0.f};
     if (active) {
-        const float4 a = *reinterpret_cast<const float4*>(dq_acc + row * D + d0);
-        const float4 c = *reinterpret_cast<const float4*>(dq_acc + row * D + kHalf + d0);
+        const float4 a = *reinterpret_cast<const float4*>(acc + row * D + d0);
+        const float4 c = *reinterpret_cast<const float4*>(acc + row * D + kHalf + d0);
         u_lo[0] = a.x * P.scale; u_lo[1] = a.y * P.scale; u_lo[2] = a.z * P.scale; u_lo[3] = a.w * P.scale;
         u_hi[0] = c.x * P.scale; u_hi[1] = c.y * P.scale; u_hi[2] = c.z * P.scale; u_hi[3] = c.w * P.scale;
+        if (P.qk_norm) {
+            load_bf16x4(x + row * D + d0, x_lo);
+            load_bf16x4(x + row * D + kHalf + d0, x_hi);
+        }
         if (P.rope) {
-            const int t = (int)((row / P.Hq) % P.T);
-            const int b = (int)(row / ((long long)P.Hq * P.T));
+            const int t = (int)((row / H) % P.T);
+            const int b = (int)(row / ((long long)H * P.T));
             const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
             const float2* cs = P.rope_cs + (size_t)pos * kHalf + d0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) rope_transpose(u_lo[i], u_hi[i], cs[i]);
-        }
-        if (P.qk_norm) {
-            load_bf16x4(q + row * D + d0, x_lo);
-            load_bf16x4(q + row * D + kHalf + d0, x_hi);
         }
     }
     if (P.qk_norm) {
@@ -227,8 +240,8 @@ __global__ void __launch_bounds__(256) k_dq_finalize(const float* __restrict__ d
         }
     }
     if (!active) return;
-    store_bf16x4(dq + row * D + d0, u_lo);
-    store_bf16x4(dq + row * D + kHalf + d0, u_hi);
+    store_bf16x4(out + row * D + d0, u_lo);
+    store_bf16x4(out + row * D + kHalf + d0, u_hi);
 }
 
 // ------------------------------------------------------------------ launchers
@@ -265,11 +278,14 @@ static cudaError_t launch_bwd_pre_d(const Problem& P, const void* o, const void*
 }
 
 template <int D>
-static cudaError_t launch_dq_finalize_d(const Problem& P, const float* dq_acc, const void* q, void* dq,
-                                        cudaStream_t st) {
-    const long long rows = (long long)P.B * P.T * P.Hq;
-    k_dq_finalize<D><<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(dq_acc, (const __nv_bfloat16*)q,
-                                                                 (__nv_bfloat16*)dq, P, rows);
+static cudaError_t launch_grad_finalize_d(const Problem& P, const float* dq_acc, const float* dk_acc, const void* q,
+                                          const void* k, void* dq, void* dk, cudaStream_t st) {
+    const long long rows_q = (long long)P.B * P.T * P.Hq;
+    const long long rows_k = (P.rope || P.qk_norm) ? (long long)P.B * P.T * P.Hkv : 0;
+    const long long rows = rows_q + rows_k;
+    k_grad_finalize<D><<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(
+        dq_acc, dk_acc, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, P,
+        rows_q, rows);
     return cudaGetLastError();
 }
 
@@ -293,8 +309,9 @@ cudaError_t launch_bwd_pre(const Problem& P, const void* o, const void* dout, fl
     CSA_DISPATCH_D(P.D, CALL)
 #undef CALL
 }
-cudaError_t launch_dq_finalize(const Problem& P, const float* dq_acc, const void* q, void* dq, cudaStream_t st) {
-#define CALL(d) launch_dq_finalize_d<d>(P, dq_acc, q, dq, st)
+cudaError_t launch_grad_finalize(const Problem& P, const float* dq_acc, const float* dk_acc, const void* q,
+                                 const void* k, void* dq, void* dk, cudaStream_t st) {
+#define CALL(d) launch_grad_finalize_d<d>(P, dq_acc, dk_acc, q, k, dq, dk, st)
     CSA_DISPATCH_D(P.D, CALL)
 #undef CALL
 }

@@ -92,4 +92,4 @@ def test_status_strings(b):
         assert b.status_string(code)
     assert b.status_string(6) == "a bounded wait inside a kernel ran out"
     assert b.kernel_names() == ["k_prep", "k_qk_prologue", "k_attn_fwd", "k_bwd_pre", "k_attn_bwd",
-                                "k_dq_finalize"]
+                                "k_grad_finalize"]
