@@ -11,11 +11,12 @@
 // One CTA owns a 128-key tile of one (b, kv head) and loops over the G query heads of the
 // group and every 128-row query tile that sees those keys, so dK and dV of the group sum in
 // TMEM without atomics.  dQ' tiles are added into an fp32 accumulator with vector reductions.
-// Warp roles (384 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer: K', V once; Q', dO tiles into a 2-stage ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 4-7   P / dS computation (thread = key row = TMEM lane), then the dK'/dV epilogue
-//   warps 8-11  dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
+//   warps 4-11  P / dS computation, two warpgroups on the same key rows (thread = key row =
+//               TMEM lane), queries [0,64) and [64,128); then the dV / dK' epilogue
+//   warps 12-15 dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
 //               k_grad_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
 // written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
@@ -92,6 +93,11 @@ __device__ __forceinline__ uint64_t ds_desc_mnmajor(uint32_t tile, int ks) {  //
     return sdesc(tile + ks * 16 * 128, 128 * 128, 1024, kLayoutSw128);
 }
 
+// TMEM column (relative to S^T) of P^T's packed bf16 pairs for the 16-query MMA K-step ks.
+// Each softmax half writes its P^T over its own first 32 S^T columns, so neither half can
+// overwrite scores the other has not read: queries [0,64) -> [0,32), [64,128) -> [64,96).
+__device__ __forceinline__ uint32_t pt_col(int ks) { return 8 * ks + (ks >= 4 ? 32 : 0); }
+
 // Queries that see key j: [lo, hi] (empty when lo > hi).
 __device__ __forceinline__ void col_bounds(const Problem& P, int b, int j, int& lo, int& hi) {
     if (j >= P.T || j < 0) {
@@ -113,7 +119,7 @@ __device__ __forceinline__ void col_bounds(const Problem& P, int b, int j, int& 
 }
 
 template <int D, bool CAP>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dq, const BwdArgs A) {
@@ -170,12 +176,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(ds_full, 128);
+        mbar_init(ds_full, 256);
         mbar_init(ds_free, 1);
         mbar_init(dq_full, 1);
         mbar_init(dq_empty, 128);
         mbar_init(acc_full, 1);
-        mbar_init(wg_sync, 128);
+        mbar_init(wg_sync, 256);
         mbar_init(drain_sync, 128);
         *abort_flag = 0;
         fence_barrier_init();
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(384, 1)
                 // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
-                    umma_ts(t_dv, t_s + ks * 8, bdesc_mnmajor<D>(sdo + s * C::TILE, ks), C::IDESC_KV,
+                    umma_ts(t_dv, t_s + pt_col(ks), bdesc_mnmajor<D>(sdo + s * C::TILE, ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
                 // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
 #pragma unroll
@@ -284,9 +290,11 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (ok) umma_commit(acc_full);
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ================= P / dS, then the dK / dV epilogue
-        const int kr = tid - 128;
+    } else if (warp >= 4 && warp < 12) {
+        // ================= P / dS, then the dK / dV epilogue.  Two warpgroups on the same key
+        // rows (TMEM lanes): `half` 0 takes queries [0, 64), half 1 queries [64, 128).
+        const int half = (warp >= 8) ? 1 : 0;
+        const int kr = tid - 128 - 128 * half;
         const int key = n * kBN + kr;
         int lo, hi;
         col_bounds(P, b, key, lo, hi);
@@ -310,8 +318,8 @@ __global__ void __launch_bounds__(384, 1)
             const int m = m_lo + it % nm;
             const int q0 = m * kBM;
             const int buf = it & 1;
-            lse_s[buf * 128 + kr] = nl2;
-            delta_s[buf * 128 + kr] = nd;
+            if (half == 0) lse_s[buf * 128 + kr] = nl2;
+            else delta_s[buf * 128 + kr] = nd;
             if (it + 1 < nit) fetch(it + 1, nl2, nd);
             mbar_arrive(wg_sync);
             ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
@@ -325,7 +333,7 @@ __global__ void __launch_bounds__(384, 1)
             const float* ls = lse_s + buf * 128;
             const float* dl = delta_s + buf * 128;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * half; c < 2 * half + 2; ++c) {
                 uint32_t sv[32], dpv[32];
                 tmem_ld32(t_s + 32 * c, sv);
                 tmem_ld32(t_dp + 32 * c, dpv);
@@ -365,7 +373,7 @@ __global__ void __launch_bounds__(384, 1)
                     dk16[e / 2] = pack_bf16x2(dd[0], dd[1]);
                     dk16[e / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
                 }
-                tmem_st16(t_s + 16 * c, pk);  // P^T (bf16) over S^T columns already read
+                tmem_st16(t_s + pt_col(2 * c), pk);  // P^T (bf16) over this half's S^T columns already read
                 // dS^T row kr, queries [32c, 32c+32): 4 chunks of 16 bytes, 128-byte swizzle
                 uint8_t* atom_row = ds_row + (c >> 1) * (128 * 128);
 #pragma unroll
@@ -387,7 +395,7 @@ __global__ void __launch_bounds__(384, 1)
             const bool row_ok = key < P.T;
             const size_t row_off = (((size_t)b * P.T + (row_ok ? key : 0)) * P.Hkv + kvh) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < (half == 0 ? D / 32 : 0); ++c) {  // dV: first half
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_base + 32 * c, v);
                 tmem_ld_wait();
@@ -408,7 +416,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t t_dk = tmem + lane_base + 128;
             const bool transform = P.rope || P.qk_norm;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < (half == 1 ? D / 32 : 0); ++c) {  // dK': second half
                 uint32_t v[32];
                 tmem_ld32(t_dk + 32 * c, v);
                 tmem_ld_wait();
@@ -432,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 12) {
         // ================= dQ' drain (thread = query row of the current tile)
         // TMEM -> registers -> fp32 tile in shared memory -> TMA reduce-add into the global
         // accumulator.  The staging space is the finished stage's Q' and dO tiles (their MMAs
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(384, 1)
         // D/16 boxes of 16 floats x 128 rows in the 64-byte swizzle.  The dQ' columns are
         // released as soon as they are read; the stage is released to the producer once the
         // reduce has read the staging.
-        const int r = tid - 256;
+        const int r = tid - 384;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_dq = tmem + lane_base + 256;  // dQ' shares the S^T columns
         constexpr int kAtoms = D / 16;                   // 8 KB each
@@ -520,7 +528,7 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.dv = static_cast<__nv_bfloat16*>(dv);
     A.nkt = (P.T + kBN - 1) / kBN;
     const int grid = A.nkt * P.B * P.Hkv;
-    k_attn_bwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, A);
+    k_attn_bwd<D, CAP><<<grid, 512, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, A);
     return cudaGetLastError();
 }
 
