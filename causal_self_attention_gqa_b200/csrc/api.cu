@@ -24,6 +24,24 @@ cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMa
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
                        float* dk_acc, void* dk, void* dv, cudaStream_t st);
 
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -222,6 +240,7 @@ Problem make_problem(const csa_params& p, int* status) {
     P.seg_end = nullptr;
     P.rope_cs = nullptr;
     P.status = status;
+    P.counters = status + 1;
     return P;
 }
 
@@ -240,7 +259,8 @@ int prepare(const csa_params* p, bool backward, const void* q, const void* k, co
     if (ws_bytes < out.L.total) return CSA_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     out.P = make_problem(*p, reinterpret_cast<int*>(w + out.L.status));
-    if (cudaMemsetAsync(w + out.L.status, 0, sizeof(int), st) != cudaSuccess) {
+    // status word and the persistent kernels' work counters start at zero
+    if (cudaMemsetAsync(w + out.L.status, 0, 4 * sizeof(int), st) != cudaSuccess) {
         cudaGetLastError();
         return CSA_ERR_CUDA;
     }

@@ -20,7 +20,7 @@
 //               k_grad_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
 // written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
-// then reuses the S^T columns.  MMA order per tile: dV, dK, dQ' of tile i, dP^T of tile
+// then reuses the S^T columns.  MMA order per tile: dV, dQ', dK' of tile i, dP^T of tile
 // i+1 (no wait on the drain), then S^T of tile i+1 once the drain has read dQ'.  dS^T goes to shared memory (128x128
 // bf16, 128-byte swizzle) where it is the K-major A operand of dK' and, read MN-major,
 // the A operand of dQ'.
@@ -176,13 +176,13 @@ __global__ void __launch_bounds__(512, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(ds_full, 256);
+        mbar_init(ds_full, 8);      // one arrival per P/dS warp
         mbar_init(ds_free, 1);
         mbar_init(dq_full, 1);
-        mbar_init(dq_empty, 128);
+        mbar_init(dq_empty, 4);     // one arrival per drain warp
         mbar_init(acc_full, 1);
-        mbar_init(wg_sync, 256);
-        mbar_init(drain_sync, 128);
+        mbar_init(wg_sync, 8);
+        mbar_init(drain_sync, 4);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -261,19 +261,20 @@ __global__ void __launch_bounds__(512, 1)
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ts(t_dv, t_s + pt_col(ks), bdesc_mnmajor<D>(sdo + s * C::TILE, ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
+                // dQ' = dS K' into the S^T columns (P^T there is consumed by the dV MMA issued
+                // just above; MMAs of one thread run in issue order).  Issued before dK' so the
+                // drain can start while the tensor core works on dK'.
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    umma_ss(t_s, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
+                umma_commit(dq_full);
                 // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ss(t_dk, ds_desc_kmajor(sds, ks), bdesc_mnmajor<D>(sq + s * C::TILE, ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
-                // dQ' = dS K' into the S^T columns (P^T there is consumed by the dV MMA issued
-                // above; MMAs of one thread run in issue order)
-#pragma unroll
-                for (int ks = 0; ks < kBN / 16; ++ks)
-                    umma_ss(t_s, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
-                umma_commit(dq_full);
                 umma_commit(&stage_empty[s]);
-                umma_commit(ds_free);
+                umma_commit(ds_free);  // dS read by dQ' and dK'; Q'/dO of this stage no longer read
                 if (it + 1 < nit) {
                     const int s1 = (it + 1) & 1, ph1 = ((it + 1) >> 1) & 1;
                     // dP^T of the next tile right away: its columns were read before ds_full
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(512, 1)
             if (half == 0) lse_s[buf * 128 + kr] = nl2;
             else delta_s[buf * 128 + kr] = nd;
             if (it + 1 < nit) fetch(it + 1, nl2, nd);
-            mbar_arrive(wg_sync);
+            warp_arrive(wg_sync);
             ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
             ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status) &&
                  mbar_wait(dp_full, it & 1, abort_flag, P.status);
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(512, 1)
             tmem_st_wait();
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(ds_full);
+            warp_arrive(ds_full);
         }
         // ---- epilogue: dV, dK of this key row (sum over the group's query heads)
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, P.status));
@@ -460,32 +461,44 @@ __global__ void __launch_bounds__(512, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
             if (!ok) break;
             tc_fence_after();
+            // staging: the first D/2 columns go to this stage's dO tile (free: dV ran before
+            // dQ'), the second half to its Q' tile, which dK' (issued after dQ') still reads
             auto atom_base = [&](int a) -> uint8_t* {
-                return (a < kAtoms / 2) ? smem + C::OFF_Q + s * C::TILE + a * 8192
-                                        : smem + C::OFF_DO + s * C::TILE + (a - kAtoms / 2) * 8192;
+                return (a < kAtoms / 2) ? smem + C::OFF_DO + s * C::TILE + a * 8192
+                                        : smem + C::OFF_Q + s * C::TILE + (a - kAtoms / 2) * 8192;
+            };
+            auto stage_atom = [&](int a, const uint32_t* v) {  // 16 floats of row r, 64-byte swizzle
+                uint8_t* row = atom_base(a) + r * 64;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4*>(row + ((j ^ ((r >> 1) & 3)) * 16)) =
+                        make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             };
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(t_dq + 32 * c, v);
+            for (int a = 0; a < kAtoms / 2; ++a) {
+                uint32_t v[16];
+                tmem_ld16(t_dq + 16 * a, v);
                 tmem_ld_wait();
                 tmem_ld_fence(v);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint8_t* row = atom_base(2 * c + half) + r * 64;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int pc = j ^ ((r >> 1) & 3);
-                        *reinterpret_cast<uint4*>(row + pc * 16) =
-                            make_uint4(v[16 * half + 4 * j], v[16 * half + 4 * j + 1], v[16 * half + 4 * j + 2],
-                                       v[16 * half + 4 * j + 3]);
-                    }
-                }
+                stage_atom(a, v);
             }
+            uint32_t hold[D / 2];
+#pragma unroll
+            for (int a = 0; a < kAtoms / 2; ++a)
+                tmem_ld16(t_dq + 16 * (kAtoms / 2 + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
+            tmem_ld_wait();
+            tmem_ld_fence(hold);
+            // dK' done (Q' of this stage free) before dQ' columns are released: phase it+1 of
+            // ds_free needs S^T of the next tile, which waits for the dq_empty arrival below,
+            // so this parity wait can never be overtaken
+            ok = __all_sync(0xffffffffu, mbar_wait(ds_free, it & 1, abort_flag, P.status));
             tc_fence_before();
-            mbar_arrive(dq_empty);  // the dQ' columns may be overwritten now
+            warp_arrive(dq_empty);  // every dQ' column has been read: the S^T columns are free
+            if (!ok) break;
+#pragma unroll
+            for (int a = 0; a < kAtoms / 2; ++a) stage_atom(kAtoms / 2 + a, hold + 16 * a);
             fence_proxy_async_smem();
-            mbar_arrive(drain_sync);
+            warp_arrive(drain_sync);
             ok = __all_sync(0xffffffffu, mbar_wait(drain_sync, it & 1, abort_flag, P.status));
             if (!ok) break;
             if (r == 0) {

@@ -1,4 +1,4 @@
-// attn_fwd.cu -- flash-style attention forward for sm_100a (TMA + tcgen05/TMEM).
+// attn_fwd.cu -- flash-style attention forward for sm_100a (TMA + tcgen05/TMEM), persistent.
 //
 // Computes, per (b, h) and query row i, O_i = sum_j softmax_j(s'_ij) v_j over the keys j
 // visible to i, and LSE_i = log sum_j exp(s'_ij) (natural log), where s'_ij is the scaled
@@ -8,15 +8,19 @@
 // evaluated online over key tiles (running max and sum, rescaling the partial output),
 // which reaches the same result as the row softmax up to rounding.
 //
-// One CTA owns up to two 128-row query tiles that read the same key/value head:
+// A work item is up to two 128-row query tiles that read the same key/value head:
 //   * G = Hq/Hkv >= 2: two query heads of one group at the same 128 positions, so both
 //     tiles see exactly the same keys and share every K/V tile;
 //   * G == 1: two consecutive 128-position tiles of one head.
+// Items are numbered heaviest first.  The grid has one CTA per SM; each CTA takes items
+// from an atomic counter until they run out, so the loads and first MMAs of the next item
+// overlap the epilogue of the current one and no CTA setup is repeated.
 // Warp roles (384 threads):
-//   warp 0      TMA producer: the two Q tiles once, then K and V tiles into a STAGES ring
+//   warp 0      producer: claims items, publishes them through a 2-slot ring, TMA-loads the
+//               two Q tiles of each item and its K/V tiles into a STAGES ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 4-7   softmax of query tile 0 (thread = row = TMEM lane)
-//   warps 8-11  softmax of query tile 1
+//   warps 4-7   softmax and epilogue of query tile 0 (thread = row = TMEM lane)
+//   warps 8-11  softmax and epilogue of query tile 1
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D).  P_i is
 // written as packed bf16 over the first 64 columns of S_i and fed to the PV MMA from TMEM.
 // MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one softmax group
@@ -27,6 +31,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "csa_internal.h"
 #include "ptx.cuh"
@@ -45,10 +51,11 @@ struct FwdCfg {
     static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + STAGES * TILE;
     static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
-    // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2]
-    static constexpr int NBAR = 1 + 3 * STAGES + 6;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
-    static constexpr int SMEM = OFF_MISC + 16;
+    // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2],
+    // o_full[2], o_empty[2], item_full[2], item_empty[2]
+    static constexpr int NBAR = 2 + 3 * STAGES + 12;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, item ring [2]
+    static constexpr int SMEM = OFF_MISC + 32;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -59,8 +66,10 @@ struct FwdArgs {
     Problem P;
     __nv_bfloat16* o;
     float* lse;
-    int nqt;    // query tiles per (b, h)
-    int pairs;  // G >= 2: head pairs per group; G == 1: tile pairs per head
+    int* counter;  // work-item counter (zeroed by the call)
+    int nqt;       // query tiles per (b, h)
+    int pairs;     // G >= 2: head pairs per group; G == 1: tile pairs per head
+    int items;     // number of work items
 };
 
 // K-major operand (rows x D, D contiguous), 16-element K step ks.
@@ -105,6 +114,49 @@ __device__ __forceinline__ float capped_log2(float raw, const Problem& P) {
     return P.softcap * 1.4426950408889634f * t;
 }
 
+// One work item, decoded identically by every role from its index.
+struct FwdItem {
+    int b, kvh, hh[2], mm[2];
+    bool two;
+    int kt_begin, nkt;
+};
+
+__device__ __forceinline__ FwdItem decode_item(const FwdArgs& A, int idx) {
+    const Problem& P = A.P;
+    FwdItem w;
+    if (P.G >= 2) {
+        const int per = P.B * P.Hkv * A.pairs;
+        const int m = A.nqt - 1 - idx / per;
+        int rem = idx % per;
+        w.b = rem / (P.Hkv * A.pairs);
+        rem %= P.Hkv * A.pairs;
+        w.kvh = rem / A.pairs;
+        const int pg = rem % A.pairs;
+        w.hh[0] = w.kvh * P.G + 2 * pg;
+        w.hh[1] = (2 * pg + 1 < P.G) ? w.hh[0] + 1 : -1;
+        w.mm[0] = w.mm[1] = m;
+    } else {
+        const int per = P.B * P.Hq;
+        const int pp = A.pairs - 1 - idx / per;
+        const int rem = idx % per;
+        w.b = rem / P.Hq;
+        w.kvh = rem % P.Hq;
+        w.hh[0] = w.hh[1] = w.kvh;
+        w.mm[0] = 2 * pp;
+        w.mm[1] = 2 * pp + 1;
+        if (w.mm[1] >= A.nqt) w.hh[1] = -1;
+    }
+    w.two = w.hh[1] >= 0;
+    // key-tile range: union over the (one or two) query tiles; bounds are monotone in q
+    int lo0, hi0, lo1, hi1;
+    row_bounds(P, w.b, w.mm[0] * kBM, lo0, hi0);
+    const int last = w.two ? w.mm[1] : w.mm[0];
+    row_bounds(P, w.b, min(last * kBM + kBM - 1, P.T - 1), lo1, hi1);
+    w.kt_begin = lo0 / kBN;
+    w.nkt = hi1 / kBN - w.kt_begin + 1;
+    return w;
+}
+
 template <int D, bool CAP>
 __global__ void __launch_bounds__(384, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -116,56 +168,20 @@ __global__ void __launch_bounds__(384, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;
-    uint64_t* v_full = bars + 1 + C::STAGES;
-    uint64_t* kv_empty = bars + 1 + 2 * C::STAGES;
-    uint64_t* s_full = bars + 1 + 3 * C::STAGES;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* o_full = s_full + 4;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* k_full = bars + 2;
+    uint64_t* v_full = bars + 2 + C::STAGES;
+    uint64_t* kv_empty = bars + 2 + 2 * C::STAGES;
+    uint64_t* s_full = bars + 2 + 3 * C::STAGES;  // [2]
+    uint64_t* p_full = s_full + 2;                 // [2]
+    uint64_t* o_full = s_full + 4;                 // [2]
+    uint64_t* o_empty = s_full + 6;                // [2]
+    uint64_t* item_full = s_full + 8;              // [2]
+    uint64_t* item_empty = s_full + 10;            // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
 
-    // ---- work item
-    int b, kvh, hh[2], mm[2];
-    {
-        const int idx = blockIdx.x;
-        if (P.G >= 2) {
-            const int per = P.B * P.Hkv * A.pairs;
-            const int m = A.nqt - 1 - idx / per;
-            int rem = idx % per;
-            b = rem / (P.Hkv * A.pairs);
-            rem %= P.Hkv * A.pairs;
-            kvh = rem / A.pairs;
-            const int pg = rem % A.pairs;
-            hh[0] = kvh * P.G + 2 * pg;
-            hh[1] = (2 * pg + 1 < P.G) ? hh[0] + 1 : -1;
-            mm[0] = mm[1] = m;
-        } else {
-            const int per = P.B * P.Hq;
-            const int pp = A.pairs - 1 - idx / per;
-            const int rem = idx % per;
-            b = rem / P.Hq;
-            kvh = rem % P.Hq;
-            hh[0] = hh[1] = kvh;
-            mm[0] = 2 * pp;
-            mm[1] = 2 * pp + 1;
-            if (mm[1] >= A.nqt) hh[1] = -1;
-        }
-    }
-    const bool two = hh[1] >= 0;
-    // key-tile range: union over the (one or two) query tiles; bounds are monotone in q
-    int kt_begin, kt_end;
-    {
-        int lo0, hi0, lo1, hi1;
-        row_bounds(P, b, mm[0] * kBM, lo0, hi0);
-        const int last = two ? mm[1] : mm[0];
-        row_bounds(P, b, min(last * kBM + kBM - 1, P.T - 1), lo1, hi1);
-        kt_begin = lo0 / kBN;
-        kt_end = hi1 / kBN;
-    }
-    const int nkt = kt_end - kt_begin + 1;
-
-    // ---- setup
     // the swizzled tiles need a 1024-byte aligned base; the condition is uniform over the CTA
     if ((smem_u32(smem) & 1023u) != 0) {
         if (tid == 0) atomicCAS(P.status, 0, CSA_ERR_LAUNCH);
@@ -173,6 +189,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (tid == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&v_full[s], 1);
@@ -180,8 +197,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
+            mbar_init(&p_full[i], 4);   // one arrival per softmax warp
             mbar_init(&o_full[i], 1);
+            mbar_init(&o_empty[i], 4);  // one arrival per softmax warp, O read out
+            mbar_init(&item_full[i], 1);
+            mbar_init(&item_empty[i], 9);  // MMA thread + 8 softmax warps
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -195,36 +215,56 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // next item index from the ring (slot n & 1); -1 ends the loop
+    auto take_item = [&](int n, int& idx) -> bool {
+        if (!mbar_wait(&item_full[n & 1], (n >> 1) & 1, abort_flag, P.status)) return false;
+        idx = item_ring[n & 1];
+        return true;
+    };
+
     if (warp == 0) {
-        // ================= TMA producer
-        if (lane == 0 && nkt > 0) {
+        // ================= producer
+        if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const uint32_t qbytes = (two ? 2 : 1) * C::TILE;
-            mbar_arrive_expect_tx(q_full, qbytes);
-            for (int i = 0; i < (two ? 2 : 1); ++i)
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_4d(&tm_q, q_full, smem + C::OFF_Q + i * C::TILE + a * kBM * C::SW, a * C::AE, hh[i],
-                                mm[i] * kBM, b);
-            for (int jj = 0; jj < nkt; ++jj) {
-                const int s = jj % C::STAGES;
-                if (jj >= C::STAGES && !mbar_wait(&kv_empty[s], ((jj / C::STAGES) - 1) & 1, abort_flag, P.status))
-                    break;
-                const int t0 = (kt_begin + jj) * kBN;
-                mbar_arrive_expect_tx(&k_full[s], C::TILE);
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_4d(&tm_k, &k_full[s], smem + C::OFF_K + s * C::TILE + a * kBM * C::SW, a * C::AE, kvh,
-                                t0, b);
-                mbar_arrive_expect_tx(&v_full[s], C::TILE);
-                for (int a = 0; a < C::NA; ++a)
-                    tma_load_4d(&tm_v, &v_full[s], smem + C::OFF_V + s * C::TILE + a * kBM * C::SW, a * C::AE, kvh,
-                                t0, b);
+            int g = 0;  // key/value tiles loaded so far by this CTA
+            for (int n = 0;; ++n) {
+                const int idx = atomicAdd(A.counter, 1);
+                const int slot = n & 1;
+                if (n >= 2 && !mbar_wait(&item_empty[slot], ((n >> 1) - 1) & 1, abort_flag, P.status)) break;
+                item_ring[slot] = (idx < A.items) ? idx : -1;
+                mbar_arrive(&item_full[slot]);
+                if (idx >= A.items) break;
+                const FwdItem w = decode_item(A, idx);
+                // Q tiles of this item once the previous item's last S MMA has read the old ones
+                if (n >= 1 && !mbar_wait(q_empty, (n - 1) & 1, abort_flag, P.status)) break;
+                mbar_arrive_expect_tx(q_full, (w.two ? 2 : 1) * C::TILE);
+                for (int i = 0; i < (w.two ? 2 : 1); ++i)
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_4d(&tm_q, q_full, smem + C::OFF_Q + i * C::TILE + a * kBM * C::SW, a * C::AE,
+                                    w.hh[i], w.mm[i] * kBM, w.b);
+                bool ok = true;
+                for (int jj = 0; jj < w.nkt; ++jj, ++g) {
+                    const int s = g % C::STAGES;
+                    if (g >= C::STAGES && !(ok = mbar_wait(&kv_empty[s], ((g / C::STAGES) - 1) & 1, abort_flag, P.status)))
+                        break;
+                    const int t0 = (w.kt_begin + jj) * kBN;
+                    mbar_arrive_expect_tx(&k_full[s], C::TILE);
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_4d(&tm_k, &k_full[s], smem + C::OFF_K + s * C::TILE + a * kBM * C::SW, a * C::AE,
+                                    w.kvh, t0, w.b);
+                    mbar_arrive_expect_tx(&v_full[s], C::TILE);
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_load_4d(&tm_v, &v_full[s], smem + C::OFF_V + s * C::TILE + a * kBM * C::SW, a * C::AE,
+                                    w.kvh, t0, w.b);
+                }
+                if (!ok) break;
             }
         }
     } else if (warp == 1) {
         // ================= MMA issuer
-        if (lane == 0 && nkt > 0) {
+        if (lane == 0) {
             const uint32_t sq = smem_u32(smem + C::OFF_Q);
             const uint32_t sk = smem_u32(smem + C::OFF_K);
             const uint32_t sv = smem_u32(smem + C::OFF_V);
@@ -243,58 +283,81 @@ __global__ void __launch_bounds__(384, 1)
                     umma_ts(d, tmem + i * 128 + ks * 8, desc_mnmajor<D>(sv + s * C::TILE, ks), C::IDESC_PV,
                             (acc || ks > 0) ? 1u : 0u);
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag, P.status) && mbar_wait(&k_full[0], 0, abort_flag, P.status);
-            if (ok) {
+            int g = 0;                // key/value tiles consumed
+            int ps[2] = {0, 0};       // steps completed per tile (p_full parity)
+            int no[2] = {0, 0};       // items completed per tile (o_full / o_empty parity)
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                int idx;
+                if (!(ok = take_item(n, idx))) break;
+                mbar_arrive(&item_empty[n & 1]);
+                if (idx < 0) break;
+                const FwdItem w = decode_item(A, idx);
+                if (!(ok = mbar_wait(q_full, n & 1, abort_flag, P.status) &&
+                           mbar_wait(&k_full[g % C::STAGES], (g / C::STAGES) & 1, abort_flag, P.status)))
+                    break;
                 tc_fence_after();
-                issue_s(0, 0);
-                if (two) issue_s(1, 0);
-            }
-            for (int jj = 0; ok && jj < nkt; ++jj) {
-                const int s = jj % C::STAGES, ph = (jj / C::STAGES) & 1;
-                const bool next = jj + 1 < nkt;
-                const int s2 = (jj + 1) % C::STAGES, ph2 = ((jj + 1) / C::STAGES) & 1;
-                ok = mbar_wait(&v_full[s], ph, abort_flag, P.status) && mbar_wait(&p_full[0], jj & 1, abort_flag, P.status);
+                issue_s(0, g % C::STAGES);
+                if (w.two) issue_s(1, g % C::STAGES);
+                if (w.nkt == 1) umma_commit(q_empty);
+                for (int jj = 0; ok && jj < w.nkt; ++jj, ++g) {
+                    const int s = g % C::STAGES, ph = (g / C::STAGES) & 1;
+                    const bool next = jj + 1 < w.nkt;
+                    const int s2 = (g + 1) % C::STAGES, ph2 = ((g + 1) / C::STAGES) & 1;
+                    for (int i = 0; i < (w.two ? 2 : 1); ++i) {
+                        ok = mbar_wait(&v_full[s], ph, abort_flag, P.status) &&
+                             mbar_wait(&p_full[i], ps[i] & 1, abort_flag, P.status);
+                        // the first PV of an item overwrites O_i: the previous epilogue must have read it
+                        if (ok && jj == 0 && no[i] > 0) ok = mbar_wait(&o_empty[i], (no[i] - 1) & 1, abort_flag, P.status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(i, s, jj > 0);
+                        ++ps[i];
+                        if (next) {
+                            if (i == 0 && !(ok = mbar_wait(&k_full[s2], ph2, abort_flag, P.status))) break;
+                            tc_fence_after();
+                            issue_s(i, s2);
+                        }
+                    }
+                    if (!ok) break;
+                    if (jj + 2 == w.nkt) umma_commit(q_empty);  // the item's last S MMAs are issued
+                    umma_commit(&kv_empty[s]);
+                }
                 if (!ok) break;
-                tc_fence_after();
-                issue_pv(0, s, jj > 0);
-                if (next) {
-                    if (!(ok = mbar_wait(&k_full[s2], ph2, abort_flag, P.status))) break;
-                    tc_fence_after();
-                    issue_s(0, s2);
+                for (int i = 0; i < (w.two ? 2 : 1); ++i) {
+                    umma_commit(&o_full[i]);
+                    ++no[i];
                 }
-                if (two) {
-                    if (!(ok = mbar_wait(&p_full[1], jj & 1, abort_flag, P.status))) break;
-                    tc_fence_after();
-                    issue_pv(1, s, jj > 0);
-                    if (next) issue_s(1, s2);
-                }
-                umma_commit(&kv_empty[s]);
-            }
-            if (ok) {
-                umma_commit(&o_full[0]);
-                if (two) umma_commit(&o_full[1]);
             }
         }
     } else if (warp >= 4) {
-        // ================= softmax, one query tile per warpgroup
+        // ================= softmax + epilogue, one query tile per warpgroup
         const int i = (warp >= 8) ? 1 : 0;
-        if (i == 0 || two) {
-            const int r = tid - 128 * (i + 1);  // row in tile == TMEM lane
-            const int h = hh[i];
-            const int q = mm[i] * kBM + r;
+        const int r = tid - 128 * (i + 1);  // row in tile == TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + i * 128;
+        const uint32_t tO = tmem + lane_base + 256 + i * 128;
+        int ps = 0;  // steps processed by this tile (s_full parity)
+        int no = 0;  // items finished by this tile (o_full parity)
+        bool ok = true;
+        for (int n = 0; ok; ++n) {
+            int idx = -1;
+            ok = __all_sync(0xffffffffu, take_item(n, idx));
+            warp_arrive(&item_empty[n & 1]);
+            if (!ok || idx < 0) break;
+            const FwdItem w = decode_item(A, idx);
+            if (i == 1 && !w.two) continue;
+            const int h = w.hh[i];
+            const int q = w.mm[i] * kBM + r;
             int lo, hi;
-            row_bounds(P, b, q, lo, hi);
-            const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-            const uint32_t tS = tmem + lane_base + i * 128;
-            const uint32_t tO = tmem + lane_base + 256 + i * 128;
+            row_bounds(P, w.b, q, lo, hi);
             float m_used = -INFINITY, l = 0.f;
-            bool ok = nkt > 0;
-            for (int jj = 0; ok && jj < nkt; ++jj) {
-                ok = mbar_wait(&s_full[i], jj & 1, abort_flag, P.status);
+            for (int jj = 0; ok && jj < w.nkt; ++jj, ++ps) {
+                ok = mbar_wait(&s_full[i], ps & 1, abort_flag, P.status);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
-                const int k0 = (kt_begin + jj) * kBN;
+                const int k0 = (w.kt_begin + jj) * kBN;
                 uint32_t raw[128];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, reinterpret_cast<uint32_t(&)[32]>(raw[32 * c]));
@@ -317,9 +380,13 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(raw[c]));
+                for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        mx4[u] = fmax3(mx4[u], __uint_as_float(raw[c + 2 * u]), __uint_as_float(raw[c + 2 * u + 1]));
+                }
                 const float xmul = CAP ? 1.0f : P.scale_log2;
-                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * xmul;
+                const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * xmul;
                 // rescale only when the running max grows by more than 2^8 (exact either way:
                 // O and l always share the same reference max)
                 const float m_new = fmaxf(m_used, mx);
@@ -330,20 +397,35 @@ __global__ void __launch_bounds__(384, 1)
                     m_used = m_new;
                 }
                 const float nbase = (m_used == -INFINITY) ? 0.f : -m_used;
-                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float2 xm2 = make_float2(xmul, xmul), nb2 = make_float2(nbase, nbase);
+                float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
+                // p = 2^(x - m): MUFU for most pairs; in tiles with no masked key (warp-uniform)
+                // one pair in four goes to the FMA pipe so both units share the work
+                auto exp_pass = [&](auto emu_tag) {
+                    constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(raw[32 * c + 2 * e]), xmul, nbase));
-                        const float p1 = ex2(fmaf(__uint_as_float(raw[32 * c + 2 * e + 1]), xmul, nbase));
-                        rs4[e & 3] += p0 + p1;
-                        pk[e] = pack_bf16x2(p0, p1);
+                        for (int e = 0; e < 16; ++e) {
+                            const float2 xv = ffma2(make_float2(__uint_as_float(raw[32 * c + 2 * e]),
+                                                                __uint_as_float(raw[32 * c + 2 * e + 1])),
+                                                    xm2, nb2);
+                            float2 pv;
+                            if (kEmu && (e & 3) == 3)
+                                pv = exp2_fma2(make_float2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f)));
+                            else
+                                pv = make_float2(ex2(xv.x), ex2(xv.y));
+                            if (e & 1) rsb = fadd2(rsb, pv);
+                            else rsa = fadd2(rsa, pv);
+                            pk[e] = pack_bf16x2(pv.x, pv.y);
+                        }
+                        tmem_st16(tS + 16 * c, pk);
                     }
-                    tmem_st16(tS + 16 * c, pk);
-                }
-                const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+                };
+                if (__all_sync(0xffffffffu, full)) exp_pass(std::true_type{});
+                else exp_pass(std::false_type{});
+                const float rs = (rsa.x + rsa.y) + (rsb.x + rsb.y);
                 l = l * alpha + rs;
                 if (jj > 0 && __any_sync(0xffffffffu, need)) {
                     // the previous PV has completed (it was issued before this S MMA)
@@ -360,34 +442,34 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&p_full[i]);
+                warp_arrive(&p_full[i]);
             }
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[i], 0, abort_flag, P.status));
-            if (ok) {
-                tc_fence_after();
-                const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-                const bool row_ok = q < P.T;
-                __nv_bfloat16* orow = A.o + (((size_t)b * P.T + (row_ok ? q : 0)) * P.Hq + h) * D;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t ov[32];
-                    tmem_ld32(tO + 32 * c, ov);
-                    tmem_ld_wait();
-                    tmem_ld_fence(ov);
-                    uint32_t pk[16];
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_full[i], no & 1, abort_flag, P.status));
+            if (!ok) break;
+            ++no;
+            tc_fence_after();
+            // O leaves TMEM first, then the next item's PV may overwrite it
+            const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+            uint32_t pk[D / 2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
-                    if (row_ok) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(tO + 32 * c, ov);
+                tmem_ld_wait();
+                tmem_ld_fence(ov);
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-                    }
-                }
-                if (row_ok)
-                    A.lse[((size_t)b * P.Hq + h) * P.T + q] =
-                        (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+                for (int e = 0; e < 16; ++e)
+                    pk[16 * c + e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+            }
+            tc_fence_before();
+            warp_arrive(&o_empty[i]);
+            if (q < P.T) {
+                uint4* dst = reinterpret_cast<uint4*>(A.o + (((size_t)w.b * P.T + q) * P.Hq + h) * D);
+#pragma unroll
+                for (int v4 = 0; v4 < D / 8; ++v4)
+                    dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                A.lse[((size_t)w.b * P.Hq + h) * P.T + q] =
+                    (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
             }
         }
     }
@@ -415,16 +497,17 @@ static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.P = P;
     A.o = static_cast<__nv_bfloat16*>(o);
     A.lse = lse;
+    A.counter = P.counters;  // cleared together with the status word by the call
     A.nqt = (P.T + kBM - 1) / kBM;
-    int items;
     if (P.G >= 2) {
         A.pairs = (P.G + 1) / 2;
-        items = P.B * P.Hkv * A.pairs * A.nqt;
+        A.items = P.B * P.Hkv * A.pairs * A.nqt;
     } else {
         A.pairs = (A.nqt + 1) / 2;
-        items = P.B * P.Hq * A.pairs;
+        A.items = P.B * P.Hq * A.pairs;
     }
-    k_attn_fwd<D, CAP><<<items, 384, C::SMEM, st>>>(tq, tk, tv, A);
+    const int grid = A.items < num_sms() ? A.items : num_sms();
+    k_attn_fwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, A);
     return cudaGetLastError();
 }
 

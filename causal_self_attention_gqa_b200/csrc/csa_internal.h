@@ -25,8 +25,13 @@ struct Problem {
     const int32_t* seg_start;  // [B, T] first index of each token's segment, or null
     const int32_t* seg_end;    // [B, T] one past its last index, or null
     const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
-    int* status;               // device status word (workspace)
+    int* status;               // device status word (workspace, or the caller's)
+    int* counters;             // [2] work-item counters of the persistent kernels (workspace,
+                               // zeroed by every call): forward, backward
 };
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
 
 // Kernel ids for the timing interface (order = csa_kernel_name()).
 enum KernelId { kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kNumKernels };

@@ -61,6 +61,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// One arrival per warp: every lane has finished its part (and its fences) at __syncwarp,
+// then lane 0 arrives.  Barriers fed this way count warps, not threads.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Named barrier over `count` threads (a warpgroup), id 1..15 (0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -229,6 +236,61 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// Packed fp32x2 arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for two values on the FMA/ALU pipes instead of MUFU (used for a share of the softmax
+// exponentials so both pipes work).  Range reduction: n = round(x) by the 1.5 * 2^23
+// addition trick, f = x - n in [-0.5, 0.5]; 2^f from a degree-4 polynomial fitted here by
+// the Remez exchange algorithm for minimax relative error on [-0.5, 0.5] (max relative
+// error 2.6e-6, far below the bf16 rounding the probabilities get); 2^n is added to the
+// exponent field with one integer multiply-add.  Valid for x in [-126, 127]: callers clamp.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    const float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float2 t = fadd2(x, make_float2(kRound, kRound));             // n + 1.5 * 2^23
+    const float2 n = fadd2(t, make_float2(-kRound, -kRound));            // n (exact)
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);                // x - n (exact)
+    float2 p = make_float2(9.570102207362652e-3f, 9.570102207362652e-3f);
+    p = ffma2(p, f, make_float2(5.591785907745361e-2f, 5.591785907745361e-2f));
+    p = ffma2(p, f, make_float2(2.40247443318367e-1f, 2.40247443318367e-1f));
+    p = ffma2(p, f, make_float2(6.931217908859253e-1f, 6.931217908859253e-1f));
+    p = ffma2(p, f, make_float2(9.999992847442627e-1f, 9.999992847442627e-1f));
+    // (bits of t) << 23 == n << 23 (mod 2^32): the constant part of t shifts out
+    return make_float2(__int_as_float(__float_as_int(t.x) * 8388608 + __float_as_int(p.x)),
+                       __int_as_float(__float_as_int(t.y) * 8388608 + __float_as_int(p.y)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     // cvt packs its first source into the upper half

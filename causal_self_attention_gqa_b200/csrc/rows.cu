@@ -115,9 +115,16 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
     const bool active = valid && lane16 < D / 8;
     const int d0 = 4 * lane16;
     float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 cs01 = make_float4(1.f, 0.f, 1.f, 0.f), cs23 = cs01;
     if (active) {
         load_bf16x4(x + d0, lo);
         load_bf16x4(x + kHalf + d0, hi);
+        if (P.rope) {  // issued together with the row loads: its latency overlaps theirs
+            const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
+            const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
+            cs01 = cs[0];
+            cs23 = cs[1];
+        }
     }
     float rs = 1.0f;
     if (P.qk_norm) {
@@ -134,14 +141,13 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
         hi[i] *= rs;
     }
     if (P.rope) {
-        const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
-        const float2* cs = P.rope_cs + (size_t)pos * kHalf + d0;
+        const float2 cs[4] = {make_float2(cs01.x, cs01.y), make_float2(cs01.z, cs01.w), make_float2(cs23.x, cs23.y),
+                              make_float2(cs23.z, cs23.w)};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float2 c = cs[i];
             const float a = lo[i], bb = hi[i];
-            lo[i] = a * c.x - bb * c.y;
-            hi[i] = bb * c.x + a * c.y;
+            lo[i] = a * cs[i].x - bb * cs[i].y;
+            hi[i] = bb * cs[i].x + a * cs[i].y;
         }
     }
     store_bf16x4(y + d0, lo);
@@ -217,9 +223,12 @@ __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__
             const int t = (int)((row / H) % P.T);
             const int b = (int)(row / ((long long)H * P.T));
             const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
-            const float2* cs = P.rope_cs + (size_t)pos * kHalf + d0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) rope_transpose(u_lo[i], u_hi[i], cs[i]);
+            const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
+            const float4 c01 = cs[0], c23 = cs[1];
+            rope_transpose(u_lo[0], u_hi[0], make_float2(c01.x, c01.y));
+            rope_transpose(u_lo[1], u_hi[1], make_float2(c01.z, c01.w));
+            rope_transpose(u_lo[2], u_hi[2], make_float2(c23.x, c23.y));
+            rope_transpose(u_lo[3], u_hi[3], make_float2(c23.z, c23.w));
         }
     }
     if (P.qk_norm) {
