@@ -76,6 +76,26 @@ def flops(w, segment_ids):
     return fwd, bwd, pairs
 
 
+def rank_workload(w, rank: int):
+    """The batch rank `rank` runs: same shape, its own seed (independent problems, weak scaling)."""
+    return w.with_(seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step: float, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's time."""
+    return flops_per_rank_step * world * steps / (ms_max * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -295,7 +315,7 @@ def main():
     from causal_self_attention_gqa_b200 import _binding as csa
 
     # every rank runs its own batch of the workload (weak scaling)
-    wr = w.with_(seed=w.seed + 7919 * rank)
+    wr = rank_workload(w, rank)
     inp = make_inputs(wr)
     seg_np = inp["segment_ids"].numpy() if inp["segment_ids"] is not None else None
     f_fwd, f_bwd, pairs = flops(wr, seg_np)
@@ -346,14 +366,9 @@ def main():
     if rc != 0:
         raise RuntimeError(f"device status after the timed region: {csa.status_string(rc)}")
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
     ms_per_step = ms_max / args.steps
-    total_flops = (f_fwd + f_bwd) * world * args.steps
-    value = total_flops / (ms_max * 1e-3) / 1e12
+    value = job_tflops(f_fwd + f_bwd, world, args.steps, ms_max)
     tokens_per_s = wr.B * wr.T * world * args.steps / (ms_max * 1e-3)
 
     # per-kernel times (library events on the launch stream, same timed region)
@@ -401,12 +416,8 @@ def main():
             hdv.copy_(gv, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": (f_fwd + f_bwd) * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": job_tflops(f_fwd + f_bwd, world, n_e2e, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e_ms / n_e2e}
 

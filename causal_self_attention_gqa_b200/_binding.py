@@ -31,7 +31,7 @@ CSA_ERR_NOT_IMPLEMENTED = 8
 # every entry point include/csa.h declares
 EXPORTED = ["csa_workspace_size", "csa_attn_fwd", "csa_attn_bwd", "csa_device_status",
             "csa_status_string", "csa_timing_enable", "csa_timing_collect", "csa_num_kernels",
-            "csa_kernel_name", "csa_attn_fwd_static_scratch"]
+            "csa_kernel_name", "csa_attn_fwd_static_scratch", "csa_selftest_bounded_wait"]
 
 
 class Params(ctypes.Structure):
@@ -52,6 +52,8 @@ _lib.csa_attn_bwd.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _
 _lib.csa_attn_bwd.restype = ctypes.c_int
 _lib.csa_attn_fwd_static_scratch.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.csa_attn_fwd_static_scratch.restype = ctypes.c_int
+_lib.csa_selftest_bounded_wait.argtypes = [_vp, ctypes.c_size_t, _vp]
+_lib.csa_selftest_bounded_wait.restype = ctypes.c_int
 _lib.csa_device_status.argtypes = [_vp, _vp]
 _lib.csa_device_status.restype = ctypes.c_int
 _lib.csa_status_string.argtypes = [ctypes.c_int]
@@ -180,6 +182,19 @@ def attn_bwd(q, k, v, o, do, lse, *, causal=True, window=0, softcap=0.0, rope_ba
 def device_status(workspace, stream=None) -> int:
     """csa_device_status: synchronises the stream, returns (and clears) the device-side status."""
     return int(_lib.csa_device_status(_ptr(workspace), _stream(stream)))
+
+
+def selftest_bounded_wait(device=None):
+    """csa_selftest_bounded_wait: runs the never-completing-wait kernel and returns
+    (status, gave_up[128], cycles[128]); status is CSA_ERR_DEVICE_TIMEOUT when every
+    bounded wait gave up as designed."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    ws = torch.zeros(2048, dtype=torch.uint8, device=dev)
+    rc = int(_lib.csa_selftest_bounded_wait(_ptr(ws), ws.numel(), _stream(None)))
+    body = ws[256:256 + 128 * 4 + 128 * 8].cpu()
+    gave_up = body[:512].view(torch.int32).tolist()
+    cycles = body[512:].view(torch.int64).tolist()
+    return rc, gave_up, cycles
 
 
 def timing_enable(on: bool) -> None:

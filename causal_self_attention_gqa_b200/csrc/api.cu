@@ -11,6 +11,8 @@
 #include "csa_internal.h"
 
 namespace csa {
+int run_selftest_wait(int* status, void* out, cudaStream_t st);
+size_t selftest_out_bytes();
 cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end, float2* rope_cs,
                         double rope_base, cudaStream_t st);
 cudaError_t launch_prologue(const Problem& P, const void* q, const void* k, void* qo, void* ko, cudaStream_t st);
@@ -352,6 +354,22 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
         return rc;
     return timed(kGradFinalize, st,
                  [&] { return launch_grad_finalize(pr.P, dq_acc, dk_acc, q, k, dq, dk, st); });
+}
+
+int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return CSA_ERR_ALIGNMENT;
+    if (workspace_bytes < 256 + selftest_out_bytes()) return CSA_ERR_WORKSPACE;
+    int rc = check_device();
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    if ((rc = run_selftest_wait(status, static_cast<uint8_t*>(workspace) + 256, st))) return rc;
+    return csa_device_status(workspace, stream);
 }
 
 int csa_device_status(void* workspace, void* stream) {

@@ -73,26 +73,6 @@ struct BwdArgs {
     int nkt;  // key tiles per (b, kv head)
 };
 
-template <int D>
-__device__ __forceinline__ uint64_t bdesc_kmajor(uint32_t tile, int ks) {
-    using C = BwdCfg<D>;
-    const int e = ks * 16;
-    return sdesc(tile + (e / C::AE) * (kBM * C::SW) + (e % C::AE) * 2, 16, 8 * C::SW, C::LAYOUT);
-}
-template <int D>
-__device__ __forceinline__ uint64_t bdesc_mnmajor(uint32_t tile, int ks) {
-    using C = BwdCfg<D>;
-    return sdesc(tile + ks * 16 * C::SW, kBM * C::SW, 8 * C::SW, C::LAYOUT);
-}
-// dS^T tile: 128 key rows x 128 query columns, 128-byte swizzle, two 64-column atoms.
-__device__ __forceinline__ uint64_t ds_desc_kmajor(uint32_t tile, int ks) {  // A of dK: M = key, K = q
-    const int e = ks * 16;
-    return sdesc(tile + (e / 64) * (128 * 128) + (e % 64) * 2, 16, 1024, kLayoutSw128);
-}
-__device__ __forceinline__ uint64_t ds_desc_mnmajor(uint32_t tile, int ks) {  // A of dQ: M = q, K = key
-    return sdesc(tile + ks * 16 * 128, 128 * 128, 1024, kLayoutSw128);
-}
-
 // TMEM column (relative to S^T) of P^T's packed bf16 pairs for the 16-query MMA K-step ks.
 // Each softmax half writes its P^T over its own first 32 S^T columns, so neither half can
 // overwrite scores the other has not read: queries [0,64) -> [0,32), [64,128) -> [64,96).
@@ -225,21 +205,32 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp == 1) {
         // ================= MMA issuer
         if (lane == 0 && nit > 0) {
-            const uint32_t sk = smem_u32(smem + C::OFF_K), sv = smem_u32(smem + C::OFF_V);
-            const uint32_t sq = smem_u32(smem + C::OFF_Q), sdo = smem_u32(smem + C::OFF_DO);
-            const uint32_t sds = smem_u32(smem + C::OFF_DS);
+            // operand descriptors, built once; each MMA adds a compile-time K-step offset
+            constexpr uint32_t kTileU = C::TILE >> 4;
+            const uint64_t dk_k = sdesc(smem_u32(smem + C::OFF_K), 16, 8 * C::SW, C::LAYOUT);   // K' as A (K-major)
+            const uint64_t dk_mn = sdesc(smem_u32(smem + C::OFF_K), kBM * C::SW, 8 * C::SW, C::LAYOUT);  // K' as B of dQ
+            const uint64_t dv_k = sdesc(smem_u32(smem + C::OFF_V), 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t dq_k = sdesc(smem_u32(smem + C::OFF_Q), 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t dq_mn = sdesc(smem_u32(smem + C::OFF_Q), kBM * C::SW, 8 * C::SW, C::LAYOUT);
+            const uint64_t ddo_k = sdesc(smem_u32(smem + C::OFF_DO), 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t ddo_mn = sdesc(smem_u32(smem + C::OFF_DO), kBM * C::SW, 8 * C::SW, C::LAYOUT);
+            const uint64_t dds_k = sdesc(smem_u32(smem + C::OFF_DS), 16, 1024, kLayoutSw128);         // dS^T, A of dK'
+            const uint64_t dds_mn = sdesc(smem_u32(smem + C::OFF_DS), 128 * 128, 1024, kLayoutSw128);  // dS, A of dQ'
+            auto kk = [](int ks) { return koff_kmajor<C::SW, kBM>(ks); };
+            auto kmn = [](int ks) { return koff_mnmajor<C::SW>(ks); };
+            auto kds = [](int ks) { return koff_kmajor<128, 128>(ks); };
             const uint32_t t_dv = tmem, t_dk = tmem + 128, t_s = tmem + 256, t_dp = tmem + 384;
             // S^T = K' Q'^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D)
             auto issue_s = [&](int st) {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_ss(t_s, bdesc_kmajor<D>(sk, ks), bdesc_kmajor<D>(sq + st * C::TILE, ks), C::IDESC_S, ks > 0);
+                    umma_ss(t_s, dk_k + kk(ks), dq_k + st * kTileU + kk(ks), C::IDESC_S, ks > 0);
                 umma_commit(s_full);
             };
             auto issue_dp = [&](int st) {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_ss(t_dp, bdesc_kmajor<D>(sv, ks), bdesc_kmajor<D>(sdo + st * C::TILE, ks), C::IDESC_S, ks > 0);
+                    umma_ss(t_dp, dv_k + kk(ks), ddo_k + st * kTileU + kk(ks), C::IDESC_S, ks > 0);
                 umma_commit(dp_full);
             };
             bool ok = mbar_wait(kv_full, 0, abort_flag, P.status) && mbar_wait(&q_full[0], 0, abort_flag, P.status);
@@ -259,19 +250,19 @@ __global__ void __launch_bounds__(512, 1)
                 // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
-                    umma_ts(t_dv, t_s + pt_col(ks), bdesc_mnmajor<D>(sdo + s * C::TILE, ks), C::IDESC_KV,
+                    umma_ts(t_dv, t_s + pt_col(ks), ddo_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
                 // dQ' = dS K' into the S^T columns (P^T there is consumed by the dV MMA issued
                 // just above; MMAs of one thread run in issue order).  Issued before dK' so the
                 // drain can start while the tensor core works on dK'.
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
-                    umma_ss(t_s, ds_desc_mnmajor(sds, ks), bdesc_mnmajor<D>(sk, ks), C::IDESC_Q, ks > 0);
+                    umma_ss(t_s, dds_mn + koff_mnmajor<128>(ks), dk_mn + kmn(ks), C::IDESC_Q, ks > 0);
                 umma_commit(dq_full);
                 // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
-                    umma_ss(t_dk, ds_desc_kmajor(sds, ks), bdesc_mnmajor<D>(sq + s * C::TILE, ks), C::IDESC_KV,
+                    umma_ss(t_dk, dds_k + kds(ks), dq_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(&stage_empty[s]);
                 umma_commit(ds_free);  // dS read by dQ' and dK'; Q'/dO of this stage no longer read

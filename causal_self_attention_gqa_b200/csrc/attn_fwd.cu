@@ -72,20 +72,6 @@ struct FwdArgs {
     int items;     // number of work items
 };
 
-// K-major operand (rows x D, D contiguous), 16-element K step ks.
-template <int D>
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int ks) {
-    using C = FwdCfg<D>;
-    const int e = ks * 16;
-    return sdesc(tile + (e / C::AE) * (kBM * C::SW) + (e % C::AE) * 2, 16, 8 * C::SW, C::LAYOUT);
-}
-// MN-major operand (rows = K index, D contiguous = N index), 16-row K step ks.
-template <int D>
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks) {
-    using C = FwdCfg<D>;
-    return sdesc(tile + ks * 16 * C::SW, kBM * C::SW, 8 * C::SW, C::LAYOUT);
-}
-
 // Keys visible to query row q: [lo, hi] (empty when lo > hi).
 __device__ __forceinline__ void row_bounds(const Problem& P, int b, int q, int& lo, int& hi) {
     if (q >= P.T || q < 0) {
@@ -265,22 +251,25 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 1) {
         // ================= MMA issuer
         if (lane == 0) {
-            const uint32_t sq = smem_u32(smem + C::OFF_Q);
-            const uint32_t sk = smem_u32(smem + C::OFF_K);
-            const uint32_t sv = smem_u32(smem + C::OFF_V);
+            // operand descriptors of the first Q tile and first K/V stage; others are offsets
+            const uint64_t dq0 = sdesc(smem_u32(smem + C::OFF_Q), 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t dk0 = sdesc(smem_u32(smem + C::OFF_K), 16, 8 * C::SW, C::LAYOUT);
+            const uint64_t dv0 = sdesc(smem_u32(smem + C::OFF_V), kBM * C::SW, 8 * C::SW, C::LAYOUT);
+            constexpr uint32_t kTileU = C::TILE >> 4;
             auto issue_s = [&](int i, int s) {
                 const uint32_t d = tmem + i * 128;
+                const uint64_t qd = dq0 + i * kTileU, kd = dk0 + s * kTileU;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_ss(d, desc_kmajor<D>(sq + i * C::TILE, ks), desc_kmajor<D>(sk + s * C::TILE, ks), C::IDESC_S,
-                            ks > 0);
+                    umma_ss(d, qd + koff_kmajor<C::SW, kBM>(ks), kd + koff_kmajor<C::SW, kBM>(ks), C::IDESC_S, ks > 0);
                 umma_commit(&s_full[i]);
             };
             auto issue_pv = [&](int i, int s, bool acc) {
                 const uint32_t d = tmem + 256 + i * 128;
+                const uint64_t vd = dv0 + s * kTileU;
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
-                    umma_ts(d, tmem + i * 128 + ks * 8, desc_mnmajor<D>(sv + s * C::TILE, ks), C::IDESC_PV,
+                    umma_ts(d, tmem + i * 128 + ks * 8, vd + koff_mnmajor<C::SW>(ks), C::IDESC_PV,
                             (acc || ks > 0) ? 1u : 0u);
             };
             int g = 0;                // key/value tiles consumed

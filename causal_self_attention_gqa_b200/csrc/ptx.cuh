@@ -223,6 +223,20 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
     return d;
 }
 
+// Descriptor start-address offsets (16-byte units) of the 16-element K step ks, so that the
+// MMA issuer builds each operand's descriptor once and only adds a compile-time constant per
+// instruction (the start-address field is the low 14 bits; shared addresses stay < 256 KB).
+//   K-major tile: ROWS rows, SW-byte swizzle rows, D split into SW/2-element atom columns.
+template <int SW, int ROWS>
+__host__ __device__ constexpr uint32_t koff_kmajor(int ks) {
+    return static_cast<uint32_t>(((16 * ks) / (SW / 2)) * (ROWS * SW) + ((16 * ks) % (SW / 2)) * 2) >> 4;
+}
+//   MN-major tile: K index along rows of SW bytes, 16 rows per step.
+template <int SW>
+__host__ __device__ constexpr uint32_t koff_mnmajor(int ks) {
+    return static_cast<uint32_t>(16 * ks * SW) >> 4;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B and an fp32 accumulator.
 // a_mn / b_mn: operand stored MN-major (M or N contiguous) instead of K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {

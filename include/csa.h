@@ -105,6 +105,17 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
  * synchronisation itself failed).  Resets the recorded status to CSA_OK. */
 int csa_device_status(void* workspace, void* stream);
 
+/* Self-test of the bounded waits every kernel relies on (failure detection without a GPU
+ * fault): launches one 128-thread CTA whose threads wait on mbarrier phases that never
+ * complete.  Each wait gives up after about a second of SM clocks, or as soon as another
+ * thread of the CTA has given up, records CSA_ERR_DEVICE_TIMEOUT in the workspace status
+ * word and returns; the CTA then exits normally.  The workspace (>= 2048 bytes, 256-byte
+ * aligned) receives the status word at offset 0 and, at offset 256, int gave_up[128]
+ * followed by long long cycles[128] (1 = that thread's wait gave up; clocks it waited).
+ * Synchronises the stream and returns the device status read back: CSA_ERR_DEVICE_TIMEOUT
+ * when the mechanism works, a host-side error code otherwise. */
+int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* csa_status_string(int code);
 
