@@ -12,16 +12,17 @@
 // group and every 128-row query tile that sees those keys, so dK and dV of the group sum in
 // TMEM without atomics.  dQ' tiles are added into an fp32 accumulator with vector reductions.
 // Warp roles (512 threads):
-//   warp 0      TMA producer: K', V once; Q', dO tiles into a 2-stage ring
+//   warp 0      TMA producer: K', V once; Q', dO tiles into a 2- or 3-stage ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 4-11  P / dS computation, two warpgroups on the same key rows (thread = key row =
 //               TMEM lane), queries [0,64) and [64,128); then the dV / dK' epilogue
 //   warps 12-15 dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
 //               k_grad_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
-// written as packed bf16 over the first 64 columns of S^T (A operand of the dV MMA); dQ'
-// then reuses the S^T columns.  MMA order per tile: dV, dQ', dK' of tile i, dP^T of tile
-// i+1 (no wait on the drain), then S^T of tile i+1 once the drain has read dQ'.  dS^T goes to shared memory (128x128
+// written as packed bf16 over S^T columns (A operand of the dV MMA); dQ' reuses the dP^T
+// columns.  MMA order per tile: dV(i), S^T(i+1), dK'(i), dQ'(i), then dP^T(i+1) once the
+// drain has read dQ' out of TMEM.  The P/dS warps compute P of tile i+1 (needs S^T only)
+// while dK', dQ' and the drain run, then dS once dP^T arrives.  dS^T goes to shared memory (128x128
 // bf16, 128-byte swizzle) where it is the K-major A operand of dK' and, read MN-major,
 // the A operand of dQ'.
 #include <cuda.h>
@@ -42,7 +43,9 @@ struct BwdCfg {
     static constexpr int NA = D / AE;
     static constexpr uint32_t LAYOUT = (SW == 128) ? kLayoutSw128 : kLayoutSw64;
     static constexpr int TILE = kBM * D * 2;
-    static constexpr int STAGES = 2;
+    // Q'/dO ring depth: a stage is refilled only after the dQ' drain has reduced out of it, so
+    // a third stage (when it fits) keeps the next tiles' loads off the critical path
+    static constexpr int STAGES = (D <= 96) ? 3 : 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = TILE;
     static constexpr int OFF_Q = 2 * TILE;
@@ -51,9 +54,9 @@ struct BwdCfg {
     static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;   // 2 x 128 fp32 (log2 units)
     static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
     static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
-    // kv_full, q_full[2], do_full[2], stage_empty[2], s_full, dp_full, ds_full, ds_free,
-    // dq_full, dq_empty, acc_full, wg_sync, drain_sync
-    static constexpr int NBAR = 16;
+    // kv_full, q_full[STAGES], do_full[STAGES], stage_empty[STAGES], s_full, dp_full, ds_full,
+    // ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync
+    static constexpr int NBAR = 1 + 3 * STAGES + 9;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -109,19 +112,20 @@ __global__ void __launch_bounds__(512, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    constexpr int NS = C::STAGES;
     uint64_t* kv_full = bars + 0;
-    uint64_t* q_full = bars + 1;       // [2]
-    uint64_t* do_full = bars + 3;      // [2]
-    uint64_t* stage_empty = bars + 5;  // [2]
-    uint64_t* s_full = bars + 7;
-    uint64_t* dp_full = bars + 8;
-    uint64_t* ds_full = bars + 9;
-    uint64_t* ds_free = bars + 10;
-    uint64_t* dq_full = bars + 11;
-    uint64_t* dq_empty = bars + 12;
-    uint64_t* acc_full = bars + 13;
-    uint64_t* wg_sync = bars + 14;     // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
-    uint64_t* drain_sync = bars + 15;  // the dQ drain warpgroup's own barrier
+    uint64_t* q_full = bars + 1;                // [NS]
+    uint64_t* do_full = bars + 1 + NS;          // [NS]
+    uint64_t* stage_empty = bars + 1 + 2 * NS;  // [NS]
+    uint64_t* s_full = bars + 1 + 3 * NS;
+    uint64_t* dp_full = s_full + 1;
+    uint64_t* ds_full = s_full + 2;
+    uint64_t* ds_free = s_full + 3;
+    uint64_t* dq_full = s_full + 4;
+    uint64_t* dq_empty = s_full + 5;
+    uint64_t* acc_full = s_full + 6;
+    uint64_t* wg_sync = s_full + 7;     // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
+    uint64_t* drain_sync = s_full + 8;  // the dQ drain warpgroup's own barrier
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     if (tid == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&do_full[s], 1);
             mbar_init(&stage_empty[s], 2);  // MMA commit + drain (staging read by the reduce)
@@ -188,8 +192,8 @@ __global__ void __launch_bounds__(512, 1)
                 tma_load_4d(&tm_v, kv_full, smem + C::OFF_V + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
             }
             for (int it = 0; it < nit; ++it) {
-                const int s = it & 1;
-                if (it >= 2 && !mbar_wait(&stage_empty[s], ((it >> 1) - 1) & 1, abort_flag, P.status)) break;
+                const int s = it % NS;
+                if (it >= NS && !mbar_wait(&stage_empty[s], ((it / NS) - 1) & 1, abort_flag, P.status)) break;
                 const int h = kvh * P.G + it / nm;
                 const int m = m_lo + it % nm;
                 mbar_arrive_expect_tx(&q_full[s], C::TILE);
@@ -244,7 +248,9 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
             for (int it = 0; ok && it < nit; ++it) {
-                const int s = it & 1;
+                const int s = it % NS;
+                const bool next = it + 1 < nit;
+                const int s1 = (it + 1) % NS, ph1 = ((it + 1) / NS) & 1;
                 if (!(ok = mbar_wait(ds_full, it & 1, abort_flag, P.status))) break;
                 tc_fence_after();
                 // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
@@ -252,32 +258,34 @@ __global__ void __launch_bounds__(512, 1)
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ts(t_dv, t_s + pt_col(ks), ddo_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
-                // dQ' = dS K' into the S^T columns (P^T there is consumed by the dV MMA issued
-                // just above; MMAs of one thread run in issue order).  Issued before dK' so the
-                // drain can start while the tensor core works on dK'.
-#pragma unroll
-                for (int ks = 0; ks < kBN / 16; ++ks)
-                    umma_ss(t_s, dds_mn + koff_mnmajor<128>(ks), dk_mn + kmn(ks), C::IDESC_Q, ks > 0);
-                umma_commit(dq_full);
+                // S^T of the next tile right behind dV (which consumed P^T from these columns;
+                // MMAs of one thread run in issue order): its P phase overlaps dK', dQ' below
+                if (next) {
+                    if (!(ok = mbar_wait(&q_full[s1], ph1, abort_flag, P.status))) break;
+                    tc_fence_after();
+                    issue_s(s1);
+                }
                 // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ss(t_dk, dds_k + kds(ks), dq_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
+                // dQ' = dS K' into the dP^T columns (read by the P/dS warps before ds_full).
+                // Issued last, so dq_full also means dV and dK' are done: the drain may stage
+                // into this stage's dO and Q' tiles as soon as it sees dq_full.
+#pragma unroll
+                for (int ks = 0; ks < kBN / 16; ++ks)
+                    umma_ss(t_dp, dds_mn + koff_mnmajor<128>(ks), dk_mn + kmn(ks), C::IDESC_Q, ks > 0);
+                umma_commit(dq_full);
                 umma_commit(&stage_empty[s]);
-                umma_commit(ds_free);  // dS read by dQ' and dK'; Q'/dO of this stage no longer read
-                if (it + 1 < nit) {
-                    const int s1 = (it + 1) & 1, ph1 = ((it + 1) >> 1) & 1;
-                    // dP^T of the next tile right away: its columns were read before ds_full
-                    if (!(ok = mbar_wait(&do_full[s1], ph1, abort_flag, P.status))) break;
-                    tc_fence_after();
-                    issue_dp(s1);
-                    // S^T of the next tile once the drain has read dQ' out of those columns
-                    if (!(ok = mbar_wait(&q_full[s1], ph1, abort_flag, P.status) &&
+                umma_commit(ds_free);  // dS read by dK' and dQ'
+                if (next) {
+                    // dP^T of the next tile once the drain has read dQ' out of those columns
+                    if (!(ok = mbar_wait(&do_full[s1], ph1, abort_flag, P.status) &&
                                mbar_wait(dq_empty, it & 1, abort_flag, P.status)))
                         break;
                     tc_fence_after();
-                    issue_s(s1);
+                    issue_dp(s1);
                 }
             }
             if (ok) umma_commit(acc_full);
@@ -315,31 +323,29 @@ __global__ void __launch_bounds__(512, 1)
             if (it + 1 < nit) fetch(it + 1, nl2, nd);
             warp_arrive(wg_sync);
             ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
-            ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status) &&
-                 mbar_wait(dp_full, it & 1, abort_flag, P.status);
-            if (ok && it > 0) ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, P.status);
+            ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             const bool full = (q0 >= lo) && (q0 + kBM - 1 <= hi);
             const float* ls = lse_s + buf * 128;
             const float* dl = delta_s + buf * 128;
-#pragma unroll 1
-            for (int c = 2 * half; c < 2 * half + 2; ++c) {
-                uint32_t sv[32], dpv[32];
+            // P phase (needs S^T only): P^T goes to TMEM for dV; P times the cap factor stays in
+            // registers as bf16 pairs (the value dS is built from once dP^T arrives)
+            uint32_t pd[2][16];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+                uint32_t sv[32];
                 tmem_ld32(t_s + 32 * c, sv);
-                tmem_ld32(t_dp + 32 * c, dpv);
                 tmem_ld_wait();
                 tmem_ld_fence(sv);
-                tmem_ld_fence(dpv);
-                uint32_t pk[16], dk16[16];
+                uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 l4 = *reinterpret_cast<const float4*>(ls + 32 * c + e);
-                    const float4 d4 = *reinterpret_cast<const float4*>(dl + 32 * c + e);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pp[4], dd[4];
+                    float pp[4], pf[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const float raw = __uint_as_float(sv[e + u]);
@@ -358,14 +364,51 @@ __global__ void __launch_bounds__(512, 1)
                             if (q < lo || q > hi) p = 0.f;
                         }
                         pp[u] = p;
-                        dd[u] = p * (__uint_as_float(dpv[e + u]) - dv4[u]) * dfac;
+                        pf[u] = p * dfac;
                     }
                     pk[e / 2] = pack_bf16x2(pp[0], pp[1]);
                     pk[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-                    dk16[e / 2] = pack_bf16x2(dd[0], dd[1]);
-                    dk16[e / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
+                    if constexpr (CAP) {
+                        pd[cc][e / 2] = pack_bf16x2(pf[0], pf[1]);
+                        pd[cc][e / 2 + 1] = pack_bf16x2(pf[2], pf[3]);
+                    } else {
+                        pd[cc][e / 2] = pk[e / 2];
+                        pd[cc][e / 2 + 1] = pk[e / 2 + 1];
+                    }
                 }
                 tmem_st16(t_s + pt_col(2 * c), pk);  // P^T (bf16) over this half's S^T columns already read
+            }
+            // dS phase: dP^T of this tile, and the dS^T buffer free (dK', dQ' of the last tile done)
+            ok = mbar_wait(dp_full, it & 1, abort_flag, P.status);
+            if (ok && it > 0) ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, P.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                tmem_st_wait();
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+                uint32_t dpv[32];
+                tmem_ld32(t_dp + 32 * c, dpv);
+                tmem_ld_wait();
+                tmem_ld_fence(dpv);
+                uint32_t dk16[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(dl + 32 * c + e);
+                    const uint32_t w0 = pd[cc][e / 2], w1 = pd[cc][e / 2 + 1];
+                    const float2 p01 = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u));
+                    const float2 p23 = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
+                    const float2 g01 = fadd2(make_float2(__uint_as_float(dpv[e]), __uint_as_float(dpv[e + 1])),
+                                             make_float2(-d4.x, -d4.y));
+                    const float2 g23 = fadd2(make_float2(__uint_as_float(dpv[e + 2]), __uint_as_float(dpv[e + 3])),
+                                             make_float2(-d4.z, -d4.w));
+                    const float2 s01 = fmul2(p01, g01), s23 = fmul2(p23, g23);
+                    dk16[e / 2] = pack_bf16x2(s01.x, s01.y);
+                    dk16[e / 2 + 1] = pack_bf16x2(s23.x, s23.y);
+                }
                 // dS^T row kr, queries [32c, 32c+32): 4 chunks of 16 bytes, 128-byte swizzle
                 uint8_t* atom_row = ds_row + (c >> 1) * (128 * 128);
 #pragma unroll
@@ -442,18 +485,18 @@ __global__ void __launch_bounds__(512, 1)
         // reduce has read the staging.
         const int r = tid - 384;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_dq = tmem + lane_base + 256;  // dQ' shares the S^T columns
+        const uint32_t t_dq = tmem + lane_base + 384;  // dQ' shares the dP^T columns
         constexpr int kAtoms = D / 16;                   // 8 KB each
         bool ok = nit > 0;
         for (int it = 0; ok && it < nit; ++it) {
-            const int s = it & 1;
+            const int s = it % NS;
             const int h = kvh * P.G + it / nm;
             const int q0 = (m_lo + it % nm) * kBM;
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
             if (!ok) break;
             tc_fence_after();
-            // staging: the first D/2 columns go to this stage's dO tile (free: dV ran before
-            // dQ'), the second half to its Q' tile, which dK' (issued after dQ') still reads
+            // staging: the first D/2 columns go to this stage's dO tile, the second half to its
+            // Q' tile; dV and dK' (their readers) finished before dQ' (dq_full)
             auto atom_base = [&](int a) -> uint8_t* {
                 return (a < kAtoms / 2) ? smem + C::OFF_DO + s * C::TILE + a * 8192
                                         : smem + C::OFF_Q + s * C::TILE + (a - kAtoms / 2) * 8192;
@@ -479,13 +522,8 @@ __global__ void __launch_bounds__(512, 1)
                 tmem_ld16(t_dq + 16 * (kAtoms / 2 + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
             tmem_ld_wait();
             tmem_ld_fence(hold);
-            // dK' done (Q' of this stage free) before dQ' columns are released: phase it+1 of
-            // ds_free needs S^T of the next tile, which waits for the dq_empty arrival below,
-            // so this parity wait can never be overtaken
-            ok = __all_sync(0xffffffffu, mbar_wait(ds_free, it & 1, abort_flag, P.status));
             tc_fence_before();
-            warp_arrive(dq_empty);  // every dQ' column has been read: the S^T columns are free
-            if (!ok) break;
+            warp_arrive(dq_empty);  // every dQ' column has been read: the dP^T columns are free
 #pragma unroll
             for (int a = 0; a < kAtoms / 2; ++a) stage_atom(kAtoms / 2 + a, hold + 16 * a);
             fence_proxy_async_smem();
