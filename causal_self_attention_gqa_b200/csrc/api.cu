@@ -235,6 +235,8 @@ Problem make_problem(const csa_params& p, int* status) {
     P.softcap = p.softcap > 0.f ? p.softcap : 0.f;
     P.scale = p.scale > 0.f ? p.scale : (float)(1.0 / sqrt((double)p.D));
     P.scale_log2 = (float)((double)P.scale * 1.4426950408889634);
+    P.cap_in = P.softcap > 0.f ? (float)((double)P.scale / (double)P.softcap) : 0.f;
+    P.cap_log2 = (float)((double)P.softcap * 1.4426950408889634);
     P.rope = p.rope_base > 0.f ? 1 : 0;
     P.qk_norm = p.qk_norm;
     P.eps = p.qk_norm_eps;

@@ -46,6 +46,9 @@ struct BwdCfg {
     // Q'/dO ring depth: a stage is refilled only after the dQ' drain has reduced out of it, so
     // a third stage (when it fits) keeps the next tiles' loads off the critical path
     static constexpr int STAGES = (D <= 96) ? 3 : 2;
+    // With two stages the Q' tile is released as soon as dK' has read it and the drain stages
+    // dQ' through the dO tile alone (two rounds of D/2 columns)
+    static constexpr bool SPLIT = STAGES == 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = TILE;
     static constexpr int OFF_Q = 2 * TILE;
@@ -54,9 +57,9 @@ struct BwdCfg {
     static constexpr int OFF_LSE = OFF_DS + 128 * 128 * 2;   // 2 x 128 fp32 (log2 units)
     static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
     static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
-    // kv_full, q_full[STAGES], do_full[STAGES], stage_empty[STAGES], s_full, dp_full, ds_full,
-    // ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync
-    static constexpr int NBAR = 1 + 3 * STAGES + 9;
+    // kv_full, q_full[STAGES], do_full[STAGES], q_empty[STAGES], do_empty[STAGES], s_full,
+    // dp_full, ds_full, ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync
+    static constexpr int NBAR = 1 + 4 * STAGES + 9;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -116,8 +119,9 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* kv_full = bars + 0;
     uint64_t* q_full = bars + 1;                // [NS]
     uint64_t* do_full = bars + 1 + NS;          // [NS]
-    uint64_t* stage_empty = bars + 1 + 2 * NS;  // [NS]
-    uint64_t* s_full = bars + 1 + 3 * NS;
+    uint64_t* q_empty = bars + 1 + 2 * NS;   // [NS]
+    uint64_t* do_empty = bars + 1 + 3 * NS;  // [NS]
+    uint64_t* s_full = bars + 1 + 4 * NS;
     uint64_t* dp_full = s_full + 1;
     uint64_t* ds_full = s_full + 2;
     uint64_t* ds_free = s_full + 3;
@@ -156,7 +160,10 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&do_full[s], 1);
-            mbar_init(&stage_empty[s], 2);  // MMA commit + drain (staging read by the reduce)
+            // MMA commit + drain (staging read by the reduce); the Q' tile holds no staging in
+            // the split scheme
+            mbar_init(&q_empty[s], C::SPLIT ? 1 : 2);
+            mbar_init(&do_empty[s], 2);
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -193,13 +200,15 @@ __global__ void __launch_bounds__(512, 1)
             }
             for (int it = 0; it < nit; ++it) {
                 const int s = it % NS;
-                if (it >= NS && !mbar_wait(&stage_empty[s], ((it / NS) - 1) & 1, abort_flag, P.status)) break;
+                const uint32_t ph = ((it / NS) - 1) & 1;
+                if (it >= NS && !mbar_wait(&q_empty[s], ph, abort_flag, P.status)) break;
                 const int h = kvh * P.G + it / nm;
                 const int m = m_lo + it % nm;
                 mbar_arrive_expect_tx(&q_full[s], C::TILE);
                 for (int a = 0; a < C::NA; ++a)
                     tma_load_4d(&tm_q, &q_full[s], smem + C::OFF_Q + s * C::TILE + a * kBM * C::SW, a * C::AE, h,
                                 m * kBM, b);
+                if (it >= NS && !mbar_wait(&do_empty[s], ph, abort_flag, P.status)) break;
                 mbar_arrive_expect_tx(&do_full[s], C::TILE);
                 for (int a = 0; a < C::NA; ++a)
                     tma_load_4d(&tm_do, &do_full[s], smem + C::OFF_DO + s * C::TILE + a * kBM * C::SW, a * C::AE, h,
@@ -270,6 +279,7 @@ __global__ void __launch_bounds__(512, 1)
                 for (int ks = 0; ks < kBM / 16; ++ks)
                     umma_ss(t_dk, dds_k + kds(ks), dq_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
+                if constexpr (C::SPLIT) umma_commit(&q_empty[s]);  // last reader of this Q' tile
                 // dQ' = dS K' into the dP^T columns (read by the P/dS warps before ds_full).
                 // Issued last, so dq_full also means dV and dK' are done: the drain may stage
                 // into this stage's dO and Q' tiles as soon as it sees dq_full.
@@ -277,7 +287,8 @@ __global__ void __launch_bounds__(512, 1)
                 for (int ks = 0; ks < kBN / 16; ++ks)
                     umma_ss(t_dp, dds_mn + koff_mnmajor<128>(ks), dk_mn + kmn(ks), C::IDESC_Q, ks > 0);
                 umma_commit(dq_full);
-                umma_commit(&stage_empty[s]);
+                umma_commit(&do_empty[s]);
+                if constexpr (!C::SPLIT) umma_commit(&q_empty[s]);
                 umma_commit(ds_free);  // dS read by dK' and dQ'
                 if (next) {
                     // dP^T of the next tile once the drain has read dQ' out of those columns
@@ -351,10 +362,8 @@ __global__ void __launch_bounds__(512, 1)
                         const float raw = __uint_as_float(sv[e + u]);
                         float p, dfac = 1.f;
                         if constexpr (CAP) {
-                            const float y = raw * P.scale / P.softcap;
-                            const float ex = ex2(y * 2.8853900817779268f);
-                            const float t = 1.0f - __fdividef(2.0f, ex + 1.0f);
-                            p = ex2(fmaf(P.softcap * kLog2e, t, -lv[u]));
+                            const float t = tanh_approx(raw * P.cap_in);
+                            p = ex2(fmaf(P.cap_log2, t, -lv[u]));
                             dfac = 1.0f - t * t;
                         } else {
                             p = ex2(fmaf(raw, P.scale_log2, -lv[u]));
@@ -478,16 +487,25 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp >= 12) {
         // ================= dQ' drain (thread = query row of the current tile)
         // TMEM -> registers -> fp32 tile in shared memory -> TMA reduce-add into the global
-        // accumulator.  The staging space is the finished stage's Q' and dO tiles (their MMAs
-        // are complete once dQ' is): together they hold exactly the 128 x D fp32 tile, as
-        // D/16 boxes of 16 floats x 128 rows in the 64-byte swizzle.  The dQ' columns are
-        // released as soon as they are read; the stage is released to the producer once the
-        // reduce has read the staging.
+        // accumulator, as boxes of 16 floats x 128 rows (8 KB) in the 64-byte swizzle.  The
+        // staging space is the finished stage's dO tile (its MMAs are complete once dQ' is),
+        // which holds D/2 fp32 columns, plus its Q' tile for the other half; in the split
+        // scheme the Q' tile is already back with the producer and the two halves go through
+        // the dO tile one after the other.  The dQ' columns are released as soon as they are
+        // read; the stage once the reduce has read the staging.
         const int r = tid - 384;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_dq = tmem + lane_base + 384;  // dQ' shares the dP^T columns
         constexpr int kAtoms = D / 16;                   // 8 KB each
+        constexpr int kHalf = kAtoms / 2;
         bool ok = nit > 0;
+        uint32_t dph = 0;  // drain_sync phase
+        auto drain_bar = [&]() -> bool {
+            warp_arrive(drain_sync);
+            const bool w = __all_sync(0xffffffffu, mbar_wait(drain_sync, dph, abort_flag, P.status));
+            dph ^= 1u;
+            return w;
+        };
         for (int it = 0; ok && it < nit; ++it) {
             const int s = it % NS;
             const int h = kvh * P.G + it / nm;
@@ -495,11 +513,11 @@ __global__ void __launch_bounds__(512, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
             if (!ok) break;
             tc_fence_after();
-            // staging: the first D/2 columns go to this stage's dO tile, the second half to its
-            // Q' tile; dV and dK' (their readers) finished before dQ' (dq_full)
+            // atom a < kHalf: this stage's dO tile; a >= kHalf: its Q' tile (dV and dK', their
+            // readers, finished before dQ' did)
             auto atom_base = [&](int a) -> uint8_t* {
-                return (a < kAtoms / 2) ? smem + C::OFF_DO + s * C::TILE + a * 8192
-                                        : smem + C::OFF_Q + s * C::TILE + (a - kAtoms / 2) * 8192;
+                return (a < kHalf) ? smem + C::OFF_DO + s * C::TILE + a * 8192
+                                   : smem + C::OFF_Q + s * C::TILE + (a - kHalf) * 8192;
             };
             auto stage_atom = [&](int a, const uint32_t* v) {  // 16 floats of row r, 64-byte swizzle
                 uint8_t* row = atom_base(a) + r * 64;
@@ -508,8 +526,13 @@ __global__ void __launch_bounds__(512, 1)
                     *reinterpret_cast<uint4*>(row + ((j ^ ((r >> 1) & 3)) * 16)) =
                         make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             };
+            auto reduce = [&](int a0, int a1, int col0) {  // atoms [a0, a1) -> columns col0 + 16 (a - a0)
+                for (int a = a0; a < a1; ++a) tma_reduce_add_4d(&tm_dq, atom_base(a), col0 + (a - a0) * 16, h, q0, b);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            };
 #pragma unroll 1
-            for (int a = 0; a < kAtoms / 2; ++a) {
+            for (int a = 0; a < kHalf; ++a) {
                 uint32_t v[16];
                 tmem_ld16(t_dq + 16 * a, v);
                 tmem_ld_wait();
@@ -518,23 +541,35 @@ __global__ void __launch_bounds__(512, 1)
             }
             uint32_t hold[D / 2];
 #pragma unroll
-            for (int a = 0; a < kAtoms / 2; ++a)
-                tmem_ld16(t_dq + 16 * (kAtoms / 2 + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
+            for (int a = 0; a < kHalf; ++a)
+                tmem_ld16(t_dq + 16 * (kHalf + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
             tmem_ld_wait();
             tmem_ld_fence(hold);
             tc_fence_before();
             warp_arrive(dq_empty);  // every dQ' column has been read: the dP^T columns are free
+            if constexpr (C::SPLIT) {
+                fence_proxy_async_smem();
+                if (!(ok = drain_bar())) break;
+                if (r == 0) reduce(0, kHalf, 0);
+                if (!(ok = drain_bar())) break;  // first half read out of the dO tile
 #pragma unroll
-            for (int a = 0; a < kAtoms / 2; ++a) stage_atom(kAtoms / 2 + a, hold + 16 * a);
-            fence_proxy_async_smem();
-            warp_arrive(drain_sync);
-            ok = __all_sync(0xffffffffu, mbar_wait(drain_sync, it & 1, abort_flag, P.status));
-            if (!ok) break;
-            if (r == 0) {
-                for (int a = 0; a < kAtoms; ++a) tma_reduce_add_4d(&tm_dq, atom_base(a), a * 16, h, q0, b);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-                mbar_arrive(&stage_empty[s]);  // second arrival: staging read, stage reusable
+                for (int a = 0; a < kHalf; ++a) stage_atom(a, hold + 16 * a);
+                fence_proxy_async_smem();
+                if (!(ok = drain_bar())) break;
+                if (r == 0) {
+                    reduce(0, kHalf, D / 2);
+                    mbar_arrive(&do_empty[s]);  // second arrival: staging read, dO tile reusable
+                }
+            } else {
+#pragma unroll
+                for (int a = 0; a < kHalf; ++a) stage_atom(kHalf + a, hold + 16 * a);
+                fence_proxy_async_smem();
+                if (!(ok = drain_bar())) break;
+                if (r == 0) {
+                    reduce(0, kAtoms, 0);
+                    mbar_arrive(&do_empty[s]);  // second arrivals: staging read, stage reusable
+                    mbar_arrive(&q_empty[s]);
+                }
             }
         }
         if (r == 0) bulk_wait_group0();

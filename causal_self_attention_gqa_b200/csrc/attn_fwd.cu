@@ -93,11 +93,8 @@ __device__ __forceinline__ void row_bounds(const Problem& P, int b, int q, int& 
 }
 
 __device__ __forceinline__ float capped_log2(float raw, const Problem& P) {
-    // s' * log2(e) with s' = c * tanh(s / c), s = scale * raw; tanh(y) = 1 - 2 / (exp(2y) + 1)
-    const float y = raw * P.scale / P.softcap;
-    const float e = ex2(y * 2.8853900817779268f);  // exp(2y)
-    const float t = 1.0f - __fdividef(2.0f, e + 1.0f);
-    return P.softcap * 1.4426950408889634f * t;
+    // s' * log2(e) with s' = c * tanh(s / c), s = scale * raw
+    return P.cap_log2 * tanh_approx(raw * P.cap_in);
 }
 
 // One work item, decoded identically by every role from its index.
@@ -401,7 +398,8 @@ __global__ void __launch_bounds__(384, 1)
                                                                 __uint_as_float(raw[32 * c + 2 * e + 1])),
                                                     xm2, nb2);
                             float2 pv;
-                            if (kEmu && (e & 3) == 3)
+                            // with the cap, tanh takes a MUFU slot too: emulate one pair in two
+                            if (kEmu && (CAP ? (e & 1) == 1 : (e & 3) == 3))
                                 pv = exp2_fma2(make_float2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f)));
                             else
                                 pv = make_float2(ex2(xv.x), ex2(xv.y));

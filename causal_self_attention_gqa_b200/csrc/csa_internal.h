@@ -18,6 +18,8 @@ struct Problem {
     int B, T, Hq, Hkv, D, G;
     int causal, window;
     float softcap;          // 0 = off
+    float cap_in;           // scale / softcap: tanh argument per raw score (cap on)
+    float cap_log2;         // softcap * log2(e): capped logit in log2 units per unit of tanh
     float scale;            // effective score scale
     float scale_log2;       // scale * log2(e)
     int rope, qk_norm;
