@@ -102,8 +102,8 @@ int check_params(const csa_params* p) {
     if (!isfinite(p->softcap) || !isfinite(p->rope_base) || !isfinite(p->scale)) return CSA_ERR_INVALID_ARG;
     if (p->qk_norm != 0 && p->qk_norm != 1) return CSA_ERR_INVALID_ARG;
     if (p->qk_norm && !(p->qk_norm_eps > 0.f && isfinite(p->qk_norm_eps))) return CSA_ERR_INVALID_ARG;
-    const double elems = (double)p->B * p->T * p->Hq * p->D;
-    if (elems * 4.0 > 9.0e18) return CSA_ERR_INVALID_ARG;
+    // row indices of the row kernels are 31-bit (multiply-shift division)
+    if ((double)p->B * p->T * (p->Hq + p->Hkv) >= 2147483648.0) return CSA_ERR_INVALID_ARG;
     return CSA_OK;
 }
 
@@ -243,6 +243,9 @@ Problem make_problem(const csa_params& p, int* status) {
     P.seg_start = nullptr;
     P.seg_end = nullptr;
     P.rope_cs = nullptr;
+    P.div_hq = make_fastdiv((uint32_t)p.Hq);
+    P.div_hkv = make_fastdiv((uint32_t)p.Hkv);
+    P.div_t = make_fastdiv((uint32_t)(p.T > 0 ? p.T : 1));
     P.status = status;
     P.counters = status + 1;
     return P;

@@ -13,6 +13,28 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 constexpr int kBM = 128;  // query rows per tile (the MMA M)
 constexpr int kBN = 128;  // keys per tile
 
+// n / d for 0 <= n < 2^31 without a division instruction: with l = ceil(log2 d) and
+// m = ceil(2^(31+l) / d) (< 2^32), floor(n m / 2^(31+l)) = floor(n / d), because the excess
+// n (m - 2^(31+l)/d) / 2^(31+l) < 2^-l <= 1/d never reaches the next multiple of 1/d.
+struct FastDiv {
+    uint32_t d, m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    FastDiv f;
+    f.d = d;
+    f.m = (uint32_t)(((1ull << (31 + l)) + d - 1) / d);
+    f.s = 31 + l;
+    return f;
+}
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+inline uint32_t fastdiv(uint32_t n, FastDiv f) {
+    return (uint32_t)(((uint64_t)n * f.m) >> f.s);
+}
+
 // Everything a kernel needs to know about the problem.
 struct Problem {
     int B, T, Hq, Hkv, D, G;
@@ -27,6 +49,7 @@ struct Problem {
     const int32_t* seg_start;  // [B, T] first index of each token's segment, or null
     const int32_t* seg_end;    // [B, T] one past its last index, or null
     const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
+    FastDiv div_hq, div_hkv, div_t;  // row -> (token, head), token -> (batch row, position)
     int* status;               // device status word (workspace, or the caller's)
     int* counters;             // [2] work-item counters of the persistent kernels (workspace,
                                // zeroed by every call): forward, backward

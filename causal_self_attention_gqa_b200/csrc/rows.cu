@@ -84,9 +84,9 @@ __global__ void __launch_bounds__(1024) k_prep(int B, int T, const int32_t* __re
         return;
     }
     if (!rope_cs) return;
-    const long long idx = (long long)(blockIdx.x - seg_blocks) * blockDim.x + threadIdx.x;
-    if (idx >= (long long)T * half) return;
-    const int t = (int)(idx / half), d = (int)(idx % half);
+    const uint32_t idx = (blockIdx.x - seg_blocks) * blockDim.x + threadIdx.x;  // T * half < 2^27
+    if (idx >= (uint32_t)T * half) return;
+    const int t = (int)(idx / half), d = (int)(idx - (uint32_t)t * half);
     const double theta = exp((-2.0 * d / (2.0 * half)) * log_base);  // base^(-2d/D)
     double s, c;
     sincos((double)t * theta, &s, &c);
@@ -98,20 +98,20 @@ template <int D>
 __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ k,
                                                      __nv_bfloat16* __restrict__ qo, __nv_bfloat16* __restrict__ ko,
-                                                     Problem P, long long rows_q, long long rows_total) {
+                                                     Problem P, uint32_t rows_q, uint32_t rows_total) {
     constexpr int kHalf = D / 2;
     const int lane16 = threadIdx.x & 15;
-    const long long row_raw = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+    const uint32_t row_raw = blockIdx.x * 16u + (threadIdx.x >> 4);
     // no early return: every lane of the warp takes part in the group shuffles below
     const bool valid = row_raw < rows_total;
-    const long long row = valid ? row_raw : 0;
+    const uint32_t row = valid ? row_raw : 0;
     const bool is_q = row < rows_q;
-    const long long r = is_q ? row : row - rows_q;
-    const int H = is_q ? P.Hq : P.Hkv;
-    const int t = (int)((r / H) % P.T);
-    const int b = (int)(r / ((long long)H * P.T));
-    const __nv_bfloat16* x = (is_q ? q : k) + r * D;
-    __nv_bfloat16* y = (is_q ? qo : ko) + r * D;
+    const uint32_t r = is_q ? row : row - rows_q;
+    const uint32_t tok = fastdiv(r, is_q ? P.div_hq : P.div_hkv);  // b * T + t
+    const uint32_t b = fastdiv(tok, P.div_t);
+    const int t = (int)(tok - b * (uint32_t)P.T);
+    const __nv_bfloat16* x = (is_q ? q : k) + (size_t)r * D;
+    __nv_bfloat16* y = (is_q ? qo : ko) + (size_t)r * D;
     const bool active = valid && lane16 < D / 8;
     const int d0 = 4 * lane16;
     float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
         load_bf16x4(x + d0, lo);
         load_bf16x4(x + kHalf + d0, hi);
         if (P.rope) {  // issued together with the row loads: its latency overlaps theirs
-            const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
+            const int pos = P.seg_start ? t - P.seg_start[tok] : t;
             const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
             cs01 = cs[0];
             cs23 = cs[1];
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
 #pragma unroll
         for (int i = 0; i < 4; ++i) ss += lo[i] * lo[i] + hi[i] * hi[i];
         ss = group16_sum(ss);
-        rs = 1.0f / sqrtf(ss / (float)D + P.eps);
+        rs = rsqrtf(ss * (1.0f / D) + P.eps);
     }
     if (!active) return;
 #pragma unroll
@@ -158,28 +158,29 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
 template <int D>
 __global__ void __launch_bounds__(256) k_bwd_pre(const __nv_bfloat16* __restrict__ o,
                                                  const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
-                                                 float* __restrict__ dq_acc, Problem P, long long rows) {
+                                                 float* __restrict__ dq_acc, Problem P, uint32_t rows) {
     const int lane16 = threadIdx.x & 15;
-    const long long row_raw = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+    const uint32_t row_raw = blockIdx.x * 16u + (threadIdx.x >> 4);
     const bool valid = row_raw < rows;  // no early return: the group shuffles need every lane
-    const long long row = valid ? row_raw : 0;
+    const uint32_t row = valid ? row_raw : 0;
     const bool active = valid && lane16 < D / 8;
     float acc = 0.f;
     if (active) {
         float a[8], g[8];
-        load_bf16x8(o + row * D + 8 * lane16, a);
-        load_bf16x8(dout + row * D + 8 * lane16, g);
+        load_bf16x8(o + (size_t)row * D + 8 * lane16, a);
+        load_bf16x8(dout + (size_t)row * D + 8 * lane16, g);
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc += a[i] * g[i];
-        float4* z = reinterpret_cast<float4*>(dq_acc + row * D + 8 * lane16);
+        float4* z = reinterpret_cast<float4*>(dq_acc + (size_t)row * D + 8 * lane16);
         z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     acc = group16_sum(acc);
     if (valid && lane16 == 0) {
-        const int h = (int)(row % P.Hq);
-        const int t = (int)((row / P.Hq) % P.T);
-        const int b = (int)(row / ((long long)P.Hq * P.T));
+        const uint32_t tok = fastdiv(row, P.div_hq);
+        const uint32_t h = row - tok * (uint32_t)P.Hq;
+        const uint32_t b = fastdiv(tok, P.div_t);
+        const uint32_t t = tok - b * (uint32_t)P.T;
         delta[((size_t)b * P.Hq + h) * P.T + t] = acc;
     }
 }
@@ -194,15 +195,14 @@ __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__
                                                        const __nv_bfloat16* __restrict__ q,
                                                        const __nv_bfloat16* __restrict__ k,
                                                        __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
-                                                       Problem P, long long rows_q, long long rows_total) {
+                                                       Problem P, uint32_t rows_q, uint32_t rows_total) {
     constexpr int kHalf = D / 2;
     const int lane16 = threadIdx.x & 15;
-    const long long row_raw = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+    const uint32_t row_raw = blockIdx.x * 16u + (threadIdx.x >> 4);
     const bool valid = row_raw < rows_total;  // no early return: the group shuffles need every lane
-    const long long row0 = valid ? row_raw : 0;
+    const uint32_t row0 = valid ? row_raw : 0;
     const bool is_q = row0 < rows_q;
-    const long long row = is_q ? row0 : row0 - rows_q;
-    const int H = is_q ? P.Hq : P.Hkv;
+    const size_t row = is_q ? row0 : row0 - rows_q;
     const float* acc = is_q ? dq_acc : dk_acc;
     const __nv_bfloat16* x = is_q ? q : k;
     __nv_bfloat16* out = is_q ? dq : dk;
@@ -220,9 +220,9 @@ __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__
             load_bf16x4(x + row * D + kHalf + d0, x_hi);
         }
         if (P.rope) {
-            const int t = (int)((row / H) % P.T);
-            const int b = (int)(row / ((long long)H * P.T));
-            const int pos = P.seg_start ? t - P.seg_start[(size_t)b * P.T + t] : t;
+            const uint32_t tok = fastdiv((uint32_t)row, is_q ? P.div_hq : P.div_hkv);  // b * T + t
+            const int t = (int)(tok - fastdiv(tok, P.div_t) * (uint32_t)P.T);
+            const int pos = P.seg_start ? t - P.seg_start[tok] : t;
             const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
             const float4 c01 = cs[0], c23 = cs[1];
             rope_transpose(u_lo[0], u_hi[0], make_float2(c01.x, c01.y));
@@ -240,8 +240,8 @@ __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__
         }
         ss = group16_sum(ss);
         dot = group16_sum(dot);
-        const float rs = 1.0f / sqrtf(ss / (float)D + P.eps);
-        const float k3 = rs * rs * rs * dot / (float)D;
+        const float rs = rsqrtf(ss * (1.0f / D) + P.eps);
+        const float k3 = rs * rs * rs * dot * (1.0f / D);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             u_lo[i] = rs * u_lo[i] - k3 * x_lo[i];
@@ -273,7 +273,7 @@ static cudaError_t launch_prologue_d(const Problem& P, const void* q, const void
     const long long rows = rows_q + (long long)P.B * P.T * P.Hkv;
     const long long blocks = (rows + 15) / 16;
     k_qk_prologue<D><<<(unsigned)blocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, rows_q, rows);
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, (uint32_t)rows_q, (uint32_t)rows);
     return cudaGetLastError();
 }
 
@@ -282,7 +282,7 @@ static cudaError_t launch_bwd_pre_d(const Problem& P, const void* o, const void*
                                     float* dq_acc, cudaStream_t st) {
     const long long rows = (long long)P.B * P.T * P.Hq;
     k_bwd_pre<D><<<(unsigned)((rows + 15) / 16), 256, 0, st>>>((const __nv_bfloat16*)o,
-                                                             (const __nv_bfloat16*)dout, delta, dq_acc, P, rows);
+                                                             (const __nv_bfloat16*)dout, delta, dq_acc, P, (uint32_t)rows);
     return cudaGetLastError();
 }
 
@@ -294,7 +294,7 @@ static cudaError_t launch_grad_finalize_d(const Problem& P, const float* dq_acc,
     const long long rows = rows_q + rows_k;
     k_grad_finalize<D><<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(
         dq_acc, dk_acc, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, P,
-        rows_q, rows);
+        (uint32_t)rows_q, (uint32_t)rows);
     return cudaGetLastError();
 }
 

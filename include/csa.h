@@ -60,7 +60,7 @@ enum {
 
 /* Problem description.  B, T >= 0 (0 is an empty problem: nothing is enqueued, CSA_OK);
  * Hq, Hkv >= 1 with Hq % Hkv == 0 (query head h uses key/value head h / (Hq / Hkv),
- * contiguous groups); D in {32, 64, 96, 128}; T <= 1 << 20. */
+ * contiguous groups); D in {32, 64, 96, 128}; T <= 1 << 20; B * T * (Hq + Hkv) < 2^31. */
 typedef struct csa_params {
     int B, T, Hq, Hkv, D;
     int causal;        /* 1: key j visible to query i only if j <= i (decoder self-attention);

@@ -46,7 +46,8 @@ def test_workspace_size(b):
     assert w - f >= 2 * 128 * 6 * 4 + 2 * 128 * 6 * 32 * 4
     for bad in (b.make_params(2, 128, 6, 4, 32), b.make_params(2, 128, 6, 6, 48),
                 b.make_params(2, 128, 6, 6, 32, qk_norm=True, qk_norm_eps=0.0),
-                b.make_params(-1, 128, 6, 6, 32), b.make_params(1, (1 << 20) + 1, 1, 1, 32)):
+                b.make_params(-1, 128, 6, 6, 32), b.make_params(1, (1 << 20) + 1, 1, 1, 32),
+                b.make_params(1024, 1 << 20, 1, 1, 32)):  # 2^31 rows: past the 31-bit row index
         assert b.workspace_size(bad, False) == 0
 
 
