@@ -19,12 +19,12 @@
 //   warps 12-15 dQ' drain: TMEM -> fp32 reductions into the global accumulator (unscaled;
 //               k_grad_finalize applies the score scale)
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
-// written as packed bf16 over S^T columns (A operand of the dV MMA); dQ' reuses the dP^T
-// columns.  MMA order per tile: dV(i), S^T(i+1), dK'(i), dQ'(i), then dP^T(i+1) once the
-// drain has read dQ' out of TMEM.  The P/dS warps compute P of tile i+1 (needs S^T only)
-// while dK', dQ' and the drain run, then dS once dP^T arrives.  dS^T goes to shared memory (128x128
-// bf16, 128-byte swizzle) where it is the K-major A operand of dK' and, read MN-major,
-// the A operand of dQ'.
+// written as packed bf16 over S^T columns (A operand of the dV MMA), dS^T likewise over
+// dP^T columns (A operand of the dK' MMA); dQ' then reuses the dP^T columns.  MMA order per
+// tile: dV(i), S^T(i+1), dK'(i), dQ'(i), then dP^T(i+1) once the drain has read dQ' out of
+// TMEM.  The P/dS warps compute P of tile i+1 (needs S^T only) while dK', dQ' and the drain
+// run, then dS once dP^T arrives.  dS^T also goes to shared memory (128x128 bf16, 128-byte
+// swizzle), where read MN-major it is the A operand of dQ'.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
@@ -227,11 +227,9 @@ __global__ void __launch_bounds__(512, 1)
             const uint64_t dq_mn = sdesc(smem_u32(smem + C::OFF_Q), kBM * C::SW, 8 * C::SW, C::LAYOUT);
             const uint64_t ddo_k = sdesc(smem_u32(smem + C::OFF_DO), 16, 8 * C::SW, C::LAYOUT);
             const uint64_t ddo_mn = sdesc(smem_u32(smem + C::OFF_DO), kBM * C::SW, 8 * C::SW, C::LAYOUT);
-            const uint64_t dds_k = sdesc(smem_u32(smem + C::OFF_DS), 16, 1024, kLayoutSw128);         // dS^T, A of dK'
             const uint64_t dds_mn = sdesc(smem_u32(smem + C::OFF_DS), 128 * 128, 1024, kLayoutSw128);  // dS, A of dQ'
             auto kk = [](int ks) { return koff_kmajor<C::SW, kBM>(ks); };
             auto kmn = [](int ks) { return koff_mnmajor<C::SW>(ks); };
-            auto kds = [](int ks) { return koff_kmajor<128, 128>(ks); };
             const uint32_t t_dv = tmem, t_dk = tmem + 128, t_s = tmem + 256, t_dp = tmem + 384;
             // S^T = K' Q'^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D)
             auto issue_s = [&](int st) {
@@ -274,22 +272,23 @@ __global__ void __launch_bounds__(512, 1)
                     tc_fence_after();
                     issue_s(s1);
                 }
-                // dK' += dS^T Q'  (A = dS^T, K-major; B = Q', MN-major)
+                // dK' += dS^T Q'  (A = dS^T from TMEM, packed over dP^T columns; B = Q', MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
-                    umma_ss(t_dk, dds_k + kds(ks), dq_mn + s * kTileU + kmn(ks), C::IDESC_KV,
+                    umma_ts(t_dk, t_dp + pt_col(ks), dq_mn + s * kTileU + kmn(ks), C::IDESC_KV,
                             (it > 0 || ks > 0) ? 1u : 0u);
                 if constexpr (C::SPLIT) umma_commit(&q_empty[s]);  // last reader of this Q' tile
-                // dQ' = dS K' into the dP^T columns (read by the P/dS warps before ds_full).
-                // Issued last, so dq_full also means dV and dK' are done: the drain may stage
-                // into this stage's dO and Q' tiles as soon as it sees dq_full.
+                // dQ' = dS K' into the dP^T columns (read by the P/dS warps before ds_full; the
+                // packed dS^T there is consumed by dK', issued before).  Issued last, so dq_full
+                // also means dV and dK' are done: the drain may stage into this stage's dO and
+                // Q' tiles as soon as it sees dq_full.
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks)
                     umma_ss(t_dp, dds_mn + koff_mnmajor<128>(ks), dk_mn + kmn(ks), C::IDESC_Q, ks > 0);
                 umma_commit(dq_full);
                 umma_commit(&do_empty[s]);
                 if constexpr (!C::SPLIT) umma_commit(&q_empty[s]);
-                umma_commit(ds_free);  // dS read by dK' and dQ'
+                umma_commit(ds_free);  // dS read by dQ'
                 if (next) {
                     // dP^T of the next tile once the drain has read dQ' out of those columns
                     if (!(ok = mbar_wait(&do_full[s1], ph1, abort_flag, P.status) &&
@@ -387,7 +386,7 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 tmem_st16(t_s + pt_col(2 * c), pk);  // P^T (bf16) over this half's S^T columns already read
             }
-            // dS phase: dP^T of this tile, and the dS^T buffer free (dK', dQ' of the last tile done)
+            // dS phase: dP^T of this tile, and the dS buffer free (dQ' of the last tile done)
             ok = mbar_wait(dp_full, it & 1, abort_flag, P.status);
             if (ok && it > 0) ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, P.status);
             ok = __all_sync(0xffffffffu, ok);
@@ -418,7 +417,10 @@ __global__ void __launch_bounds__(512, 1)
                     dk16[e / 2] = pack_bf16x2(s01.x, s01.y);
                     dk16[e / 2 + 1] = pack_bf16x2(s23.x, s23.y);
                 }
+                // dS^T (bf16) over this half's dP^T columns already read: A operand of dK'
+                tmem_st16(t_dp + pt_col(2 * c), dk16);
                 // dS^T row kr, queries [32c, 32c+32): 4 chunks of 16 bytes, 128-byte swizzle
+                // (read MN-major as the A operand of dQ')
                 uint8_t* atom_row = ds_row + (c >> 1) * (128 * 128);
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
@@ -531,23 +533,24 @@ __global__ void __launch_bounds__(512, 1)
                 bulk_commit_group();
                 bulk_wait_group_read0();
             };
-#pragma unroll 1
-            for (int a = 0; a < kHalf; ++a) {
-                uint32_t v[16];
-                tmem_ld16(t_dq + 16 * a, v);
-                tmem_ld_wait();
-                tmem_ld_fence(v);
-                stage_atom(a, v);
-            }
-            uint32_t hold[D / 2];
-#pragma unroll
-            for (int a = 0; a < kHalf; ++a)
-                tmem_ld16(t_dq + 16 * (kHalf + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
-            tmem_ld_wait();
-            tmem_ld_fence(hold);
-            tc_fence_before();
-            warp_arrive(dq_empty);  // every dQ' column has been read: the dP^T columns are free
             if constexpr (C::SPLIT) {
+                // first half straight into the dO tile, second half held in registers
+#pragma unroll 1
+                for (int a = 0; a < kHalf; ++a) {
+                    uint32_t v[16];
+                    tmem_ld16(t_dq + 16 * a, v);
+                    tmem_ld_wait();
+                    tmem_ld_fence(v);
+                    stage_atom(a, v);
+                }
+                uint32_t hold[D / 2];
+#pragma unroll
+                for (int a = 0; a < kHalf; ++a)
+                    tmem_ld16(t_dq + 16 * (kHalf + a), reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
+                tmem_ld_wait();
+                tmem_ld_fence(hold);
+                tc_fence_before();
+                warp_arrive(dq_empty);  // every dQ' column has been read: the dP^T columns are free
                 fence_proxy_async_smem();
                 if (!(ok = drain_bar())) break;
                 if (r == 0) reduce(0, kHalf, 0);
@@ -561,8 +564,18 @@ __global__ void __launch_bounds__(512, 1)
                     mbar_arrive(&do_empty[s]);  // second arrival: staging read, dO tile reusable
                 }
             } else {
+                // the whole row in registers first: the dQ' columns (which the next dP^T MMA
+                // waits for) are released after one TMEM read, before any staging
+                uint32_t hold[D];
 #pragma unroll
-                for (int a = 0; a < kHalf; ++a) stage_atom(kHalf + a, hold + 16 * a);
+                for (int a = 0; a < kAtoms; ++a)
+                    tmem_ld16(t_dq + 16 * a, reinterpret_cast<uint32_t(&)[16]>(hold[16 * a]));
+                tmem_ld_wait();
+                tmem_ld_fence(hold);
+                tc_fence_before();
+                warp_arrive(dq_empty);  // every dQ' column has been read: the dP^T columns are free
+#pragma unroll
+                for (int a = 0; a < kAtoms; ++a) stage_atom(a, hold + 16 * a);
                 fence_proxy_async_smem();
                 if (!(ok = drain_bar())) break;
                 if (r == 0) {

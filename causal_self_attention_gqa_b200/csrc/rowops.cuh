@@ -1,18 +1,11 @@
 // rowops.cuh -- small per-row helpers shared by the row kernels and the attention
-// kernels' epilogues: bf16 vector loads/stores, 16-lane group sums, transposed RoPE.
+// kernels' epilogues: bf16 vector loads/stores, lane-group sums, transposed RoPE.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace csa {
 
-__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* p, float (&f)[4]) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-    f[0] = __low2float(a); f[1] = __high2float(a);
-    f[2] = __low2float(b); f[3] = __high2float(b);
-}
 __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8]) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -23,6 +16,13 @@ __device__ __forceinline__ void load_bf16x8(const __nv_bfloat16* p, float (&f)[8
         f[2 * i + 1] = __high2float(h);
     }
 }
+__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* p, float (&f)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    f[0] = __low2float(a); f[1] = __high2float(a);
+    f[2] = __low2float(b); f[3] = __high2float(b);
+}
 __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, const float (&f)[4]) {
     const __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
     const __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
@@ -31,9 +31,20 @@ __device__ __forceinline__ void store_bf16x4(__nv_bfloat16* p, const float (&f)[
     u.y = *reinterpret_cast<const uint32_t*>(&b);
     *reinterpret_cast<uint2*>(p) = u;
 }
-__device__ __forceinline__ float group16_sum(float v) {
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* p, const float (&f)[8]) {
+    uint32_t w[4];
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, 16);
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+// Sum over aligned groups of GS lanes (GS a power of two <= 32).
+template <int GS>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = GS / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, GS);
     return v;
 }
 // Transpose of the rotate-half rotation by phi (i.e. rotation by -phi) applied to a

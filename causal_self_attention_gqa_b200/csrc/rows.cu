@@ -10,8 +10,9 @@
 // nanogpt-jax-181m model card ("Architecture"); positions restart at each packed segment
 // (same section, "RoPE frequencies are computed from packed segment positions").
 //
-// Row kernels use a group of 16 lanes per [.., D] row; lane l < D/8 owns the 4 rotation
-// pairs (d, d + D/2) for d in [4l, 4l + 4), so a rotation never crosses lanes.
+// Row kernels give each [.., D] row an aligned group of lanes; a lane owns whole rotation
+// pairs (d, d + D/2), so a rotation never crosses lanes.  The finalize uses 16-lane groups
+// with 4 pairs per lane (it holds twice the data per pair, and 16-byte lanes cost it occupancy).
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -94,14 +95,25 @@ __global__ void __launch_bounds__(1024) k_prep(int B, int T, const int32_t* __re
 }
 
 // ------------------------------------------------------------------ q/k prologue
+// Row geometry of the prologue: a lane owns the 8 rotation pairs
+// (d, d + D/2) for d in [8g, 8g + 8), so its loads and stores are 16 bytes wide; the D/16
+// lanes of a row form an aligned group of GS lanes (a power of two; D = 96 leaves 2 of 8 idle).
+template <int D>
+struct RowGeom {
+    static constexpr int LPR = D / 16;
+    static constexpr int GS = (LPR <= 2) ? 2 : (LPR <= 4 ? 4 : 8);
+    static constexpr int ROWS = 256 / GS;  // rows per 256-thread block
+};
+
 template <int D>
 __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ k,
                                                      __nv_bfloat16* __restrict__ qo, __nv_bfloat16* __restrict__ ko,
                                                      Problem P, uint32_t rows_q, uint32_t rows_total) {
+    using G = RowGeom<D>;
     constexpr int kHalf = D / 2;
-    const int lane16 = threadIdx.x & 15;
-    const uint32_t row_raw = blockIdx.x * 16u + (threadIdx.x >> 4);
+    const int g = threadIdx.x & (G::GS - 1);
+    const uint32_t row_raw = blockIdx.x * (uint32_t)G::ROWS + threadIdx.x / G::GS;
     // no early return: every lane of the warp takes part in the group shuffles below
     const bool valid = row_raw < rows_total;
     const uint32_t row = valid ? row_raw : 0;
@@ -112,46 +124,50 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
     const int t = (int)(tok - b * (uint32_t)P.T);
     const __nv_bfloat16* x = (is_q ? q : k) + (size_t)r * D;
     __nv_bfloat16* y = (is_q ? qo : ko) + (size_t)r * D;
-    const bool active = valid && lane16 < D / 8;
-    const int d0 = 4 * lane16;
-    float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
-    float4 cs01 = make_float4(1.f, 0.f, 1.f, 0.f), cs23 = cs01;
+    const bool active = valid && g < G::LPR;
+    const int d0 = 8 * g;
+    float lo[8], hi[8];
+    float4 cs[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cs[i] = make_float4(1.f, 0.f, 1.f, 0.f);
     if (active) {
-        load_bf16x4(x + d0, lo);
-        load_bf16x4(x + kHalf + d0, hi);
+        load_bf16x8(x + d0, lo);
+        load_bf16x8(x + kHalf + d0, hi);
         if (P.rope) {  // issued together with the row loads: its latency overlaps theirs
             const int pos = P.seg_start ? t - P.seg_start[tok] : t;
-            const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
-            cs01 = cs[0];
-            cs23 = cs[1];
+            const float4* c = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cs[i] = c[i];
         }
     }
     float rs = 1.0f;
     if (P.qk_norm) {
         float ss = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) ss += lo[i] * lo[i] + hi[i] * hi[i];
-        ss = group16_sum(ss);
+        for (int i = 0; i < 8; ++i) ss += lo[i] * lo[i] + hi[i] * hi[i];
+        ss = group_sum<G::GS>(ss);
         rs = rsqrtf(ss * (1.0f / D) + P.eps);
     }
     if (!active) return;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
         lo[i] *= rs;
         hi[i] *= rs;
     }
     if (P.rope) {
-        const float2 cs[4] = {make_float2(cs01.x, cs01.y), make_float2(cs01.z, cs01.w), make_float2(cs23.x, cs23.y),
-                              make_float2(cs23.z, cs23.w)};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 8; ++i) {
+            const float c = (i & 1) ? cs[i / 2].z : cs[i / 2].x;
+            const float sn = (i & 1) ? cs[i / 2].w : cs[i / 2].y;
             const float a = lo[i], bb = hi[i];
-            lo[i] = a * cs[i].x - bb * cs[i].y;
-            hi[i] = bb * cs[i].x + a * cs[i].y;
+            lo[i] = a * c - bb * sn;
+            hi[i] = bb * c + a * sn;
         }
     }
-    store_bf16x4(y + d0, lo);
-    store_bf16x4(y + kHalf + d0, hi);
+    store_bf16x8(y + d0, lo);
+    store_bf16x8(y + kHalf + d0, hi);
 }
 
 // ------------------------------------------------------------------ backward preprocess
@@ -175,7 +191,7 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const __nv_bfloat16* __restrict
         z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    acc = group16_sum(acc);
+    acc = group_sum<16>(acc);
     if (valid && lane16 == 0) {
         const uint32_t tok = fastdiv(row, P.div_hq);
         const uint32_t h = row - tok * (uint32_t)P.Hq;
@@ -238,8 +254,8 @@ __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__
             ss += x_lo[i] * x_lo[i] + x_hi[i] * x_hi[i];
             dot += u_lo[i] * x_lo[i] + u_hi[i] * x_hi[i];
         }
-        ss = group16_sum(ss);
-        dot = group16_sum(dot);
+        ss = group_sum<16>(ss);
+        dot = group_sum<16>(dot);
         const float rs = rsqrtf(ss * (1.0f / D) + P.eps);
         const float k3 = rs * rs * rs * dot * (1.0f / D);
 #pragma unroll
@@ -271,7 +287,7 @@ static cudaError_t launch_prologue_d(const Problem& P, const void* q, const void
                                      cudaStream_t st) {
     const long long rows_q = (long long)P.B * P.T * P.Hq;
     const long long rows = rows_q + (long long)P.B * P.T * P.Hkv;
-    const long long blocks = (rows + 15) / 16;
+    const long long blocks = (rows + RowGeom<D>::ROWS - 1) / RowGeom<D>::ROWS;
     k_qk_prologue<D><<<(unsigned)blocks, 256, 0, st>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, (uint32_t)rows_q, (uint32_t)rows);
     return cudaGetLastError();
