@@ -5,8 +5,10 @@
                     [--workload NAME]
 
 A step is one pass of the whole path over one batch: csa_attn_fwd (segment bounds / RoPE
-table, QK-norm+RoPE prologue, flash forward) then csa_attn_bwd (prologue recompute,
-delta preprocess, flash backward, dQ finalize), inputs resident in HBM.  The default
+table, QK-norm+RoPE prologue, flash forward) then csa_attn_bwd_after_fwd (delta
+preprocess, flash backward, dQ/dK finalize; it reads the forward's q', k' from the shared
+workspace, as a training step would, instead of recomputing the prologue), inputs resident
+in HBM.  The default
 workload is the 181M-model GQA shape (B=16, T=2048, 8 query / 4 KV heads, head dim 96,
 RoPE, QK-norm), the largest of the five shapes.  FLOPs are algorithmic: only the
 (query, key) pairs the mask keeps count, 4*D per pair per head forward, 10*D backward.
@@ -275,7 +277,7 @@ def profile_step(w):
     ws = csa.workspace_for(q, k, True, **kw)
     for _ in range(2):
         o, lse = csa.attn_fwd(q, k, v, segment_ids=seg, workspace=ws, **kw)
-        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, **kw)
+        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, after_fwd=True, **kw)
     torch.cuda.synchronize()
     rc = csa.device_status(ws)
     print(json.dumps({"profile_step": w.name, "B": w.B, "status": rc}))
@@ -331,7 +333,8 @@ def main():
 
     def step():
         csa.attn_fwd(q, k, v, segment_ids=seg, out=o, lse=lse, workspace=ws, **kw)
-        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, dq=dq, dk=dk, dv=dv, workspace=ws, **kw)
+        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, dq=dq, dk=dk, dv=dv, workspace=ws, after_fwd=True,
+                     **kw)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -408,7 +411,8 @@ def main():
             ddo = hdo.to(dev, non_blocking=True)
             dseg = hseg.to(dev, non_blocking=True) if hseg is not None else None
             oo, ll = csa.attn_fwd(dq_, dk_, dv_, segment_ids=dseg, workspace=ws, **kw)
-            gq, gk, gv = csa.attn_bwd(dq_, dk_, dv_, oo, ddo, ll, segment_ids=dseg, workspace=ws, **kw)
+            gq, gk, gv = csa.attn_bwd(dq_, dk_, dv_, oo, ddo, ll, segment_ids=dseg, workspace=ws, after_fwd=True,
+                                      **kw)
             ho.copy_(oo, non_blocking=True)
             hlse.copy_(ll, non_blocking=True)
             hdq.copy_(gq, non_blocking=True)

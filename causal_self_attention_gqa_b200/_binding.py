@@ -31,7 +31,8 @@ CSA_ERR_NOT_IMPLEMENTED = 8
 # every entry point include/csa.h declares
 EXPORTED = ["csa_workspace_size", "csa_attn_fwd", "csa_attn_bwd", "csa_device_status",
             "csa_status_string", "csa_timing_enable", "csa_timing_collect", "csa_num_kernels",
-            "csa_kernel_name", "csa_attn_fwd_static_scratch", "csa_selftest_bounded_wait"]
+            "csa_kernel_name", "csa_attn_fwd_static_scratch", "csa_selftest_bounded_wait",
+            "csa_attn_bwd_after_fwd"]
 
 
 class Params(ctypes.Structure):
@@ -50,6 +51,9 @@ _lib.csa_attn_fwd.restype = ctypes.c_int
 _lib.csa_attn_bwd.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                               ctypes.c_size_t, _vp]
 _lib.csa_attn_bwd.restype = ctypes.c_int
+_lib.csa_attn_bwd_after_fwd.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp, ctypes.c_size_t, _vp]
+_lib.csa_attn_bwd_after_fwd.restype = ctypes.c_int
 _lib.csa_attn_fwd_static_scratch.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.csa_attn_fwd_static_scratch.restype = ctypes.c_int
 _lib.csa_selftest_bounded_wait.argtypes = [_vp, ctypes.c_size_t, _vp]
@@ -153,8 +157,10 @@ def attn_fwd(q, k, v, *, causal=True, window=0, softcap=0.0, rope_base=0.0, qk_n
 
 def attn_bwd(q, k, v, o, do, lse, *, causal=True, window=0, softcap=0.0, rope_base=0.0, qk_norm=False,
              qk_norm_eps=1e-6, scale=0.0, segment_ids=None, dq=None, dk=None, dv=None, workspace=None,
-             stream=None):
-    """csa_attn_bwd: dq, dk, dv (bf16) = gradients w.r.t. the raw q, k, v."""
+             stream=None, after_fwd=False):
+    """csa_attn_bwd: dq, dk, dv (bf16) = gradients w.r.t. the raw q, k, v.  after_fwd=True calls
+    csa_attn_bwd_after_fwd instead, which reuses q', k' from `workspace` (it must be the one the
+    matching attn_fwd call used, untouched since)."""
     opts = dict(causal=causal, window=window, softcap=softcap, rope_base=rope_base, qk_norm=qk_norm,
                 qk_norm_eps=qk_norm_eps, scale=scale)
     B, T, Hq, D = q.shape
@@ -170,12 +176,15 @@ def attn_bwd(q, k, v, o, do, lse, *, causal=True, window=0, softcap=0.0, rope_ba
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
+        if after_fwd:
+            raise ValueError("after_fwd needs the workspace of the matching attn_fwd call")
         workspace = workspace_for(q, k, True, **opts)
-    rc = _lib.csa_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(seg),
-                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-                           workspace.numel() * workspace.element_size(), _stream(stream))
+    fn = _lib.csa_attn_bwd_after_fwd if after_fwd else _lib.csa_attn_bwd
+    rc = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(seg),
+            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream))
     if rc != CSA_OK:
-        raise CsaError(rc, "csa_attn_bwd")
+        raise CsaError(rc, "csa_attn_bwd_after_fwd" if after_fwd else "csa_attn_bwd")
     return dq, dk, dv
 
 

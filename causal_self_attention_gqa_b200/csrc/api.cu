@@ -259,8 +259,10 @@ struct Prepared {
     const void* qk_k;
 };
 
+// reuse: the forward already left the segment bounds, the RoPE table and q', k' in the same
+// workspace (same layout: the backward only appends); nothing is launched but the reset.
 int prepare(const csa_params* p, bool backward, const void* q, const void* k, const int32_t* seg, void* ws,
-            size_t ws_bytes, cudaStream_t st, Prepared& out) {
+            size_t ws_bytes, cudaStream_t st, Prepared& out, bool reuse = false) {
     const bool has_seg = seg != nullptr;
     out.L = layout(*p, backward, has_seg);
     if (ws_bytes < out.L.total) return CSA_ERR_WORKSPACE;
@@ -277,6 +279,11 @@ int prepare(const csa_params* p, bool backward, const void* q, const void* k, co
     out.P.seg_start = ss;
     out.P.seg_end = se;
     out.P.rope_cs = rope;
+    if (reuse) {
+        out.qk_q = needs_prologue(*p) ? static_cast<const void*>(w + out.L.qp) : q;
+        out.qk_k = needs_prologue(*p) ? static_cast<const void*>(w + out.L.kp) : k;
+        return CSA_OK;
+    }
     if (has_seg || rope) {
         const int rc = timed(kPrep, st, [&] { return launch_prep(out.P, seg, ss, se, rope, p->rope_base, st); });
         if (rc) return rc;
@@ -328,9 +335,13 @@ int csa_attn_fwd(const csa_params* p, const void* q, const void* k, const void* 
     return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, o, lse, st); });
 }
 
-int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o, const void* dout,
-                 const float* lse, const int32_t* segment_ids, void* dq, void* dk, void* dv, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace csa {
+namespace {
+int attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, const int32_t* segment_ids, void* dq, void* dk, void* dv, void* workspace,
+             size_t workspace_bytes, void* stream, bool reuse) {
     int rc = check_params(p);
     if (rc) return rc;
     if (p->B == 0 || p->T == 0) return CSA_OK;
@@ -343,7 +354,7 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
     if ((rc = check_device())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared pr;
-    if ((rc = prepare(p, true, q, k, segment_ids, workspace, workspace_bytes, st, pr))) return rc;
+    if ((rc = prepare(p, true, q, k, segment_ids, workspace, workspace_bytes, st, pr, reuse))) return rc;
     uint8_t* w = static_cast<uint8_t*>(workspace);
     float* delta = reinterpret_cast<float*>(w + pr.L.delta);
     float* dq_acc = reinterpret_cast<float*>(w + pr.L.dq_acc);
@@ -359,6 +370,22 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
         return rc;
     return timed(kGradFinalize, st,
                  [&] { return launch_grad_finalize(pr.P, dq_acc, dk_acc, q, k, dq, dk, st); });
+}
+}  // namespace
+}  // namespace csa
+
+extern "C" {
+
+int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, const int32_t* segment_ids, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    return attn_bwd(p, q, k, v, o, dout, lse, segment_ids, dq, dk, dv, workspace, workspace_bytes, stream, false);
+}
+
+int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, const int32_t* segment_ids, void* dq, void* dk,
+                           void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_bwd(p, q, k, v, o, dout, lse, segment_ids, dq, dk, dv, workspace, workspace_bytes, stream, true);
 }
 
 int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {

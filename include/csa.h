@@ -100,6 +100,18 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
                  const void* dout, const float* lse, const int32_t* segment_ids, void* dq, void* dk,
                  void* dv, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward that reuses what the forward left in the workspace: the normalised and rotated
+ * q', k' (QK-norm / RoPE on), the segment bounds and the RoPE table, so no prologue runs
+ * (a training step computes q', k' once, in its forward).  Same arguments and results as
+ * csa_attn_bwd.  Contract: the workspace (sized with for_backward = 1) was passed to
+ * csa_attn_fwd with the same *p, q, k and segment_ids, on the same stream, and nothing has
+ * written to it since.  The library cannot check this; a broken contract gives wrong
+ * gradients (every access stays inside the workspace), never a fault. */
+int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, const void* v,
+                           const void* o, const void* dout, const float* lse,
+                           const int32_t* segment_ids, void* dq, void* dk, void* dv,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last call that used it (CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA when the
  * synchronisation itself failed).  Resets the recorded status to CSA_OK. */

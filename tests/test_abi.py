@@ -77,6 +77,15 @@ def test_invalid_arguments_are_rejected_before_any_device_work(b):
     assert _call_fwd(b, good, ws=0x10080) == b.CSA_ERR_ALIGNMENT
     assert _call_fwd(b, good, nws=100) == b.CSA_ERR_WORKSPACE
     assert _call_bwd(b, b.make_params(2, 128, 6, 5, 32)) == b.CSA_ERR_INVALID_ARG
+    # the reuse entry point runs the same host checks before touching the workspace
+    q, k, v, o, do, lse, dq, dk, dv = [0x1000 * (i + 1) for i in range(9)]
+    after = b.lib.csa_attn_bwd_after_fwd
+    assert after(ctypes.byref(b.make_params(2, 128, 6, 5, 32)), q, k, v, o, do, lse, None, dq, dk, dv, 0x10000,
+                 1 << 30, None) == b.CSA_ERR_INVALID_ARG
+    assert after(ctypes.byref(good), q, k, v, o, do, lse, None, dq, dk, dv, 0x10001, 1 << 30,
+                 None) == b.CSA_ERR_ALIGNMENT
+    assert after(ctypes.byref(good), q, k, v, o, do, lse, None, dq, dk, dv, 0x10000, 16,
+                 None) == b.CSA_ERR_WORKSPACE
     ptrs = [0x1000 * (i + 1) for i in range(9)]
     ptrs[4] = 0x5004  # dout misaligned
     assert _call_bwd(b, good, ptrs) == b.CSA_ERR_ALIGNMENT

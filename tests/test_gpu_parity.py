@@ -40,7 +40,7 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
 
 
-def run_gpu(csa, inp, opts, backward=True):
+def run_gpu(csa, inp, opts, backward=True, after_fwd=False):
     dev = torch.device("cuda:0")
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     seg = inp["segment_ids"].to(dev) if inp["segment_ids"] is not None else None
@@ -49,7 +49,7 @@ def run_gpu(csa, inp, opts, backward=True):
     out = dict(o=o, lse=lse)
     if backward:
         do = inp["do"].to(dev)
-        dq, dk, dv = csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, **opts)
+        dq, dk, dv = csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, workspace=ws, after_fwd=after_fwd, **opts)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert csa.device_status(ws) == 0
@@ -112,6 +112,21 @@ def test_small_shapes_match_oracle(csa, ora, case):
     w, inp = _small(B, T, Hq, Hkv, D, seed=7 + T + D, seg=seg, **opts)
     kw = dict(w.options())
     gpu = run_gpu(csa, inp, kw)
+    ref_o, ref_lse = ora.attn_fwd(inp["q"], inp["k"], inp["v"], segment_ids=inp["segment_ids"], **kw)
+    ref_g = ora.attn_bwd(inp["q"], inp["k"], inp["v"], inp["do"], segment_ids=inp["segment_ids"], **kw)
+    check(gpu, ref_o, ref_lse, ref_g)
+
+
+@pytest.mark.parametrize("case", [SMALL[i] for i in (2, 8, 10, 13, 17)],
+                         ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}x{c[3]}D{c[4]}"
+                         + "".join(f"-{k}{v}" for k, v in c[5].items()) + ("-seg" if c[6] else ""))
+def test_backward_after_forward_reuses_the_workspace(csa, ora, case):
+    """csa_attn_bwd_after_fwd (q', k', segment bounds and RoPE table from the forward's
+    workspace, no prologue) against the oracle: with and without norm / RoPE / segments."""
+    B, T, Hq, Hkv, D, opts, seg = case
+    w, inp = _small(B, T, Hq, Hkv, D, seed=11 + T + D, seg=seg, **opts)
+    kw = dict(w.options())
+    gpu = run_gpu(csa, inp, kw, after_fwd=True)
     ref_o, ref_lse = ora.attn_fwd(inp["q"], inp["k"], inp["v"], segment_ids=inp["segment_ids"], **kw)
     ref_g = ora.attn_bwd(inp["q"], inp["k"], inp["v"], inp["do"], segment_ids=inp["segment_ids"], **kw)
     check(gpu, ref_o, ref_lse, ref_g)
