@@ -23,8 +23,8 @@ cudaError_t launch_grad_finalize(const Problem& P, const float* dq_acc, const fl
 cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                        float* lse, cudaStream_t st);
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
-                       float* dk_acc, void* dk, void* dv, cudaStream_t st);
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                       const float* lse, const float* delta, float* dq_acc, cudaStream_t st);
 
 int num_sms() {
     static int cache[64] = {0};
@@ -360,13 +360,17 @@ int attn_bwd(const csa_params* p, const void* q, const void* k, const void* v, c
     float* dq_acc = reinterpret_cast<float*>(w + pr.L.dq_acc);
     float* dk_acc = needs_prologue(*p) ? reinterpret_cast<float*>(w + pr.L.dk_acc) : nullptr;
     if ((rc = timed(kBwdPre, st, [&] { return launch_bwd_pre(pr.P, o, dout, delta, dq_acc, st); }))) return rc;
-    CUtensorMap tq, tk, tv, tdo, tdq;
+    // dK leaves the kernel as raw fp32 sums (finalize applies scale, RoPE^T and the norm
+    // backward) when QK-norm or RoPE is on, else as bf16 scale * dK'
+    CUtensorMap tq, tk, tv, tdo, tdq, tdv, tdk;
     if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
         !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&tdo, dout, p->B, p->T, p->Hq, p->D) ||
-        !make_map_f32(&tdq, dq_acc, p->B, p->T, p->Hq, p->D))
+        !make_map_f32(&tdq, dq_acc, p->B, p->T, p->Hq, p->D) || !make_map(&tdv, dv, p->B, p->T, p->Hkv, p->D) ||
+        !(dk_acc ? make_map_f32(&tdk, dk_acc, p->B, p->T, p->Hkv, p->D) : make_map(&tdk, dk, p->B, p->T, p->Hkv, p->D)))
         return CSA_ERR_CUDA;
-    if ((rc = timed(kBwd, st,
-                    [&] { return launch_bwd(pr.P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st); })))
+    if ((rc = timed(kBwd, st, [&] {
+             return launch_bwd(pr.P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st);
+         })))
         return rc;
     return timed(kGradFinalize, st,
                  [&] { return launch_grad_finalize(pr.P, dq_acc, dk_acc, q, k, dq, dk, st); });

@@ -58,8 +58,8 @@ struct BwdCfg {
     static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
     static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
     // kv_full, q_full[STAGES], do_full[STAGES], q_empty[STAGES], do_empty[STAGES], s_full,
-    // dp_full, ds_full, ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync
-    static constexpr int NBAR = 1 + 4 * STAGES + 9;
+    // dp_full, ds_full, ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync, epi_sync[2]
+    static constexpr int NBAR = 1 + 4 * STAGES + 11;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -73,9 +73,6 @@ struct BwdArgs {
     const float* lse;      // [B, Hq, T] natural log
     const float* delta;    // [B, Hq, T]
     float* dq_acc;         // [B, T, Hq, D] fp32, zeroed
-    float* dk_acc;         // [B, T, Hkv, D] fp32 raw dK' (QK-norm or RoPE on), else unused
-    __nv_bfloat16* dk;
-    __nv_bfloat16* dv;
     int nkt;  // key tiles per (b, kv head)
 };
 
@@ -108,7 +105,8 @@ template <int D, bool CAP>
 __global__ void __launch_bounds__(512, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_dq, const BwdArgs A) {
+               const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dv,
+               const __grid_constant__ CUtensorMap tm_dk, const BwdArgs A) {
     using C = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const Problem& P = A.P;
@@ -130,6 +128,7 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* acc_full = s_full + 6;
     uint64_t* wg_sync = s_full + 7;     // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
     uint64_t* drain_sync = s_full + 8;  // the dQ drain warpgroup's own barrier
+    uint64_t* epi_sync = s_full + 9;    // [2] each P/dS half's epilogue staging is complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -174,6 +173,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(acc_full, 1);
         mbar_init(wg_sync, 8);
         mbar_init(drain_sync, 4);
+        mbar_init(&epi_sync[0], 4);
+        mbar_init(&epi_sync[1], 4);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -434,56 +435,71 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_before();
             warp_arrive(ds_full);
         }
-        // ---- epilogue: dV, dK of this key row (sum over the group's query heads)
+        // ---- epilogue: dV, dK of this key tile (sums over the group's query heads).  Each half
+        // stages its tile in shared memory that no MMA reads any more (V tile for dV; K tile,
+        // then the dS buffer, for dK) in the layout of a TMA box, and one thread stores it with
+        // tiled TMA stores (rows past T are not written).
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, P.status));
         if (ok) {
             tc_fence_after();
-            const bool row_ok = key < P.T;
-            const size_t row_off = (((size_t)b * P.T + (row_ok ? key : 0)) * P.Hkv + kvh) * D;
+            const bool transform = P.rope || P.qk_norm;
+            // 32 bf16 values (16 words) of row kr at element d0 of a bf16 tile (TMA box layout)
+            auto stage_bf16 = [&](uint8_t* tile, int d0, const uint32_t* w) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int de = d0 + 8 * q;
+                    const int a = de / C::AE, j = (de % C::AE) / 8;
+                    const int swz = (C::SW == 128) ? (kr & 7) : ((kr >> 1) & 3);
+                    *reinterpret_cast<uint4*>(tile + a * (kBM * C::SW) + kr * C::SW + ((j ^ swz) * 16)) =
+                        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                }
+            };
+            // fp32 atoms of 16 columns x 128 rows (64-byte swizzle): the K tile holds D/32 of
+            // them, the dS buffer the rest
+            auto f32_atom = [&](int t) -> uint8_t* {
+                return (t < D / 32) ? smem + C::OFF_K + t * 8192 : smem + C::OFF_DS + (t - D / 32) * 8192;
+            };
+            const uint32_t t_acc = tmem + lane_base + (half == 0 ? 0 : 128);
+            const float sc = (half == 1 && !transform) ? P.scale : 1.0f;
 #pragma unroll 1
-            for (int c = 0; c < (half == 0 ? D / 32 : 0); ++c) {  // dV: first half
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_base + 32 * c, v);
+                tmem_ld32(t_acc + 32 * c, v);
                 tmem_ld_wait();
                 tmem_ld_fence(v);
-                if (row_ok) {
-                    uint4* dst = reinterpret_cast<uint4*>(A.dv + row_off + 32 * c);
+                if (half == 1 && transform) {  // raw fp32 dK' for the finalize kernel
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * v4]), __uint_as_float(v[8 * v4 + 1])),
-                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 2]), __uint_as_float(v[8 * v4 + 3])),
-                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 4]), __uint_as_float(v[8 * v4 + 5])),
-                                             pack_bf16x2(__uint_as_float(v[8 * v4 + 6]), __uint_as_float(v[8 * v4 + 7])));
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint8_t* row = f32_atom(2 * c + h2) + kr * 64;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4*>(row + ((j ^ ((kr >> 1) & 3)) * 16)) =
+                                make_uint4(v[16 * h2 + 4 * j], v[16 * h2 + 4 * j + 1], v[16 * h2 + 4 * j + 2],
+                                           v[16 * h2 + 4 * j + 3]);
+                    }
+                } else {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
+                    stage_bf16(smem + (half == 0 ? C::OFF_V : C::OFF_K), 32 * c, w);
                 }
             }
-            // dK': with QK-norm or RoPE the raw fp32 sum goes to the workspace and the
-            // finalize kernel applies scale, RoPE^T and the RMSNorm backward (a bandwidth-bound
-            // pass); without them dK = scale * dK' is written here.
-            const uint32_t t_dk = tmem + lane_base + 128;
-            const bool transform = P.rope || P.qk_norm;
-#pragma unroll 1
-            for (int c = 0; c < (half == 1 ? D / 32 : 0); ++c) {  // dK': second half
-                uint32_t v[32];
-                tmem_ld32(t_dk + 32 * c, v);
-                tmem_ld_wait();
-                tmem_ld_fence(v);
-                if (!row_ok) continue;
-                if (transform) {
-                    uint4* dst = reinterpret_cast<uint4*>(A.dk_acc + row_off + 32 * c);
-#pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        dst[v4] = make_uint4(v[4 * v4], v[4 * v4 + 1], v[4 * v4 + 2], v[4 * v4 + 3]);
+            fence_proxy_async_smem();
+            warp_arrive(&epi_sync[half]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&epi_sync[half], 0, abort_flag, P.status));
+            if (ok && kr == 0) {
+                if (half == 0) {
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_store_4d(&tm_dv, smem + C::OFF_V + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
+                } else if (transform) {
+                    for (int t = 0; t < D / 16; ++t) tma_store_4d(&tm_dk, f32_atom(t), t * 16, kvh, n * kBN, b);
                 } else {
-                    uint4* dst = reinterpret_cast<uint4*>(A.dk + row_off + 32 * c);
-                    const float sc = P.scale;
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * v4]) * sc, __uint_as_float(v[8 * v4 + 1]) * sc),
-                            pack_bf16x2(__uint_as_float(v[8 * v4 + 2]) * sc, __uint_as_float(v[8 * v4 + 3]) * sc),
-                            pack_bf16x2(__uint_as_float(v[8 * v4 + 4]) * sc, __uint_as_float(v[8 * v4 + 5]) * sc),
-                            pack_bf16x2(__uint_as_float(v[8 * v4 + 6]) * sc, __uint_as_float(v[8 * v4 + 7]) * sc));
+                    for (int a = 0; a < C::NA; ++a)
+                        tma_store_4d(&tm_dk, smem + C::OFF_K + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
                 }
+                bulk_commit_group();
+                bulk_wait_group0();
             }
         }
     } else if (warp >= 12) {
@@ -598,8 +614,8 @@ __global__ void __launch_bounds__(512, 1)
 
 template <int D, bool CAP>
 static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
-                                float* dk_acc, void* dk, void* dv, cudaStream_t st) {
+                                const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                                const float* lse, const float* delta, float* dq_acc, cudaStream_t st) {
     using C = BwdCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -613,33 +629,33 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.lse = lse;
     A.delta = delta;
     A.dq_acc = dq_acc;
-    A.dk_acc = dk_acc;
-    A.dk = static_cast<__nv_bfloat16*>(dk);
-    A.dv = static_cast<__nv_bfloat16*>(dv);
     A.nkt = (P.T + kBN - 1) / kBN;
     const int grid = A.nkt * P.B * P.Hkv;
-    k_attn_bwd<D, CAP><<<grid, 512, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, A);
+    k_attn_bwd<D, CAP><<<grid, 512, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, tdv, tdk, A);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc,
-                                float* dk_acc, void* dk, void* dv, cudaStream_t st) {
-    return (P.softcap > 0.f) ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st)
-                             : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
+                                const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                                const float* lse, const float* delta, float* dq_acc, cudaStream_t st) {
+    return (P.softcap > 0.f)
+               ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st)
+               : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st);
 }
 
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, const CUtensorMap& tdq, const float* lse, const float* delta, float* dq_acc, float* dk_acc,
-                       void* dk, void* dv, cudaStream_t st) {
+                       const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
+                       const float* lse, const float* delta, float* dq_acc, cudaStream_t st) {
+#define CSA_BWD(d) launch_bwd_d<d>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st)
     switch (P.D) {
-        case 32: return launch_bwd_d<32>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
-        case 64: return launch_bwd_d<64>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
-        case 96: return launch_bwd_d<96>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
-        case 128: return launch_bwd_d<128>(P, tq, tk, tv, tdo, tdq, lse, delta, dq_acc, dk_acc, dk, dv, st);
+        case 32: return CSA_BWD(32);
+        case 64: return CSA_BWD(64);
+        case 96: return CSA_BWD(96);
+        case 128: return CSA_BWD(128);
         default: return cudaErrorInvalidValue;
     }
+#undef CSA_BWD
 }
 
 }  // namespace csa

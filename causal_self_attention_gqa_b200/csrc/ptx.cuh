@@ -99,6 +99,14 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
         "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(src))
         : "memory");
 }
+// Tiled TMA store (shared -> global) of one box; rows past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group"
+        " [%0, {%1, %2, %3, %4}], [%5];" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(src))
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk group has finished READING its shared-memory source.
 __device__ __forceinline__ void bulk_wait_group_read0() {
