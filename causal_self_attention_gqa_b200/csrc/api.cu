@@ -20,8 +20,8 @@ cudaError_t launch_bwd_pre(const Problem& P, const void* o, const void* dout, fl
                            cudaStream_t st);
 cudaError_t launch_grad_finalize(const Problem& P, const float* dq_acc, const float* dk_acc, const void* q,
                                  const void* k, void* dq, void* dk, cudaStream_t st);
-cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                       float* lse, cudaStream_t st);
+cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, float* lse, cudaStream_t st);
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
                        const float* lse, const float* delta, float* dq_acc, cudaStream_t st);
@@ -328,11 +328,11 @@ int csa_attn_fwd(const csa_params* p, const void* q, const void* k, const void* 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Prepared pr;
     if ((rc = prepare(p, false, q, k, segment_ids, workspace, workspace_bytes, st, pr))) return rc;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
-        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D))
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&to, o, p->B, p->T, p->Hq, p->D))
         return CSA_ERR_CUDA;
-    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, o, lse, st); });
+    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, to, lse, st); });
 }
 
 }  // extern "C"
@@ -539,9 +539,9 @@ extern "C" int csa_attn_fwd_static_scratch(const csa_params* p, const void* q, c
         }
         pr.P.status = device_status;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_map(&tq, pr.qk_q, p->B, p->T, p->Hq, p->D) || !make_map(&tk, pr.qk_k, p->B, p->T, p->Hkv, p->D) ||
-        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D))
+        !make_map(&tv, v, p->B, p->T, p->Hkv, p->D) || !make_map(&to, o, p->B, p->T, p->Hq, p->D))
         return CSA_ERR_CUDA;
-    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, o, lse, st); });
+    return timed(kFwd, st, [&] { return launch_fwd(pr.P, tq, tk, tv, to, lse, st); });
 }

@@ -50,10 +50,12 @@ struct FwdCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = 2 * TILE;
     static constexpr int OFF_V = OFF_K + STAGES * TILE;
-    static constexpr int OFF_BAR = OFF_V + STAGES * TILE;
+    static constexpr int OFF_O = OFF_V + STAGES * TILE;  // O staging for the TMA store
+    static constexpr int OFF_BAR = OFF_O + TILE;
     // barriers: q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2],
     // o_full[2], o_empty[2], item_full[2], item_empty[2]
-    static constexpr int NBAR = 2 + 3 * STAGES + 12;
+    // o_turn[2] (staging hand-off between the two warpgroups), ep_sync[2]
+    static constexpr int NBAR = 2 + 3 * STAGES + 16;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, item ring [2]
     static constexpr int SMEM = OFF_MISC + 32;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
@@ -64,7 +66,6 @@ struct FwdCfg {
 
 struct FwdArgs {
     Problem P;
-    __nv_bfloat16* o;
     float* lse;
     int* counter;  // work-item counter (zeroed by the call)
     int nqt;       // query tiles per (b, h)
@@ -143,7 +144,8 @@ __device__ __forceinline__ FwdItem decode_item(const FwdArgs& A, int idx) {
 template <int D, bool CAP>
 __global__ void __launch_bounds__(384, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdArgs A) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const FwdArgs A) {
     using C = FwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const Problem& P = A.P;
@@ -161,6 +163,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* o_empty = s_full + 6;                // [2]
     uint64_t* item_full = s_full + 8;              // [2]
     uint64_t* item_empty = s_full + 10;            // [2]
+    uint64_t* o_turn = s_full + 12;                // [2] warpgroup i is done with the O staging
+    uint64_t* ep_sync = s_full + 14;               // [2] warpgroup i has staged its O tile
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
@@ -185,6 +189,8 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&o_empty[i], 4);  // one arrival per softmax warp, O read out
             mbar_init(&item_full[i], 1);
             mbar_init(&item_empty[i], 9);  // MMA thread + 8 softmax warps
+            mbar_init(&o_turn[i], 1);
+            mbar_init(&ep_sync[i], 4);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -325,6 +331,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t tO = tmem + lane_base + 256 + i * 128;
         int ps = 0;  // steps processed by this tile (s_full parity)
         int no = 0;  // items finished by this tile (o_full parity)
+        int nt = 0;  // O-staging turns taken (warpgroup 0 goes first in every item)
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int idx = -1;
@@ -332,7 +339,16 @@ __global__ void __launch_bounds__(384, 1)
             warp_arrive(&item_empty[n & 1]);
             if (!ok || idx < 0) break;
             const FwdItem w = decode_item(A, idx);
-            if (i == 1 && !w.two) continue;
+            if (i == 1 && !w.two) {
+                // no second tile in this item: pass the staging turn straight back
+                if (r == 0) {
+                    ok = mbar_wait(&o_turn[0], nt & 1, abort_flag, P.status);
+                    if (ok) mbar_arrive(&o_turn[1]);
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                ++nt;
+                continue;
+            }
             const int h = w.hh[i];
             const int q = w.mm[i] * kBM + r;
             int lo, hi;
@@ -450,15 +466,39 @@ __global__ void __launch_bounds__(384, 1)
             }
             tc_fence_before();
             warp_arrive(&o_empty[i]);
-            if (q < P.T) {
-                uint4* dst = reinterpret_cast<uint4*>(A.o + (((size_t)w.b * P.T + q) * P.Hq + h) * D);
-#pragma unroll
-                for (int v4 = 0; v4 < D / 8; ++v4)
-                    dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if (q < P.T)
                 A.lse[((size_t)w.b * P.Hq + h) * P.T + q] =
                     (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+            // O goes out through one shared staging tile (TMA box layout) and tiled TMA stores;
+            // the two warpgroups take turns, warpgroup 0 first
+            if (i == 0) {
+                if (nt > 0) ok = mbar_wait(&o_turn[1], (nt - 1) & 1, abort_flag, P.status);
+            } else {
+                ok = mbar_wait(&o_turn[0], nt & 1, abort_flag, P.status);
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            ++nt;
+#pragma unroll
+            for (int v4 = 0; v4 < D / 8; ++v4) {
+                const int a = (8 * v4) / C::AE, j = ((8 * v4) % C::AE) / 8;
+                const int swz = (C::SW == 128) ? (r & 7) : ((r >> 1) & 3);
+                *reinterpret_cast<uint4*>(smem + C::OFF_O + a * (kBM * C::SW) + r * C::SW + ((j ^ swz) * 16)) =
+                    make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            }
+            fence_proxy_async_smem();
+            warp_arrive(&ep_sync[i]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&ep_sync[i], (no - 1) & 1, abort_flag, P.status));
+            if (!ok) break;
+            if (r == 0) {
+                for (int a = 0; a < C::NA; ++a)
+                    tma_store_4d(&tm_o, smem + C::OFF_O + a * kBM * C::SW, a * C::AE, h, w.mm[i] * kBM, w.b);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(&o_turn[i]);  // staging read: the other warpgroup's turn
             }
         }
+        if (r == 0) bulk_wait_group0();
     }
 
     tc_fence_before();
@@ -471,7 +511,7 @@ __global__ void __launch_bounds__(384, 1)
 
 template <int D, bool CAP>
 static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                void* o, float* lse, cudaStream_t st) {
+                                const CUtensorMap& to, float* lse, cudaStream_t st) {
     using C = FwdCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -482,7 +522,6 @@ static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const
     }
     FwdArgs A;
     A.P = P;
-    A.o = static_cast<__nv_bfloat16*>(o);
     A.lse = lse;
     A.counter = P.counters;  // cleared together with the status word by the call
     A.nqt = (P.T + kBM - 1) / kBM;
@@ -494,24 +533,24 @@ static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const
         A.items = P.B * P.Hq * A.pairs;
     }
     const int grid = A.items < num_sms() ? A.items : num_sms();
-    k_attn_fwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, A);
+    k_attn_fwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, to, A);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                void* o, float* lse, cudaStream_t st) {
-    return (P.softcap > 0.f) ? launch_fwd_cap<D, true>(P, tq, tk, tv, o, lse, st)
-                             : launch_fwd_cap<D, false>(P, tq, tk, tv, o, lse, st);
+                                const CUtensorMap& to, float* lse, cudaStream_t st) {
+    return (P.softcap > 0.f) ? launch_fwd_cap<D, true>(P, tq, tk, tv, to, lse, st)
+                             : launch_fwd_cap<D, false>(P, tq, tk, tv, to, lse, st);
 }
 
-cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                       float* lse, cudaStream_t st) {
+cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, float* lse, cudaStream_t st) {
     switch (P.D) {
-        case 32: return launch_fwd_d<32>(P, tq, tk, tv, o, lse, st);
-        case 64: return launch_fwd_d<64>(P, tq, tk, tv, o, lse, st);
-        case 96: return launch_fwd_d<96>(P, tq, tk, tv, o, lse, st);
-        case 128: return launch_fwd_d<128>(P, tq, tk, tv, o, lse, st);
+        case 32: return launch_fwd_d<32>(P, tq, tk, tv, to, lse, st);
+        case 64: return launch_fwd_d<64>(P, tq, tk, tv, to, lse, st);
+        case 96: return launch_fwd_d<96>(P, tq, tk, tv, to, lse, st);
+        case 128: return launch_fwd_d<128>(P, tq, tk, tv, to, lse, st);
         default: return cudaErrorInvalidValue;
     }
 }
