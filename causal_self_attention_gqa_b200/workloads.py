@@ -51,7 +51,9 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads, in order; seed = 1000 + index.
+# The five benchmark-defined workloads, in order, then the short-window layer of an SSSL stack
+# (the 181M shape with a window of T/2 that binds on unpacked rows: three of every four layers
+# in a short-short-short-long pattern run it); seed = 1000 + index.
 WORKLOADS = [
     Workload("pr1_mha_T128_D32", B=2, T=128, Hq=6, Hkv=6, D=32, seed=1000),
     Workload("minigpt_T128_D32_rope_qknorm", B=32, T=128, Hq=6, Hkv=6, D=32,
@@ -62,6 +64,8 @@ WORKLOADS = [
              rope_base=10000.0, qk_norm=True, seed=1003),
     Workload("packed_sft_gqa6x3_T2048_D128_win1024", B=8, T=2048, Hq=6, Hkv=3, D=128,
              rope_base=10000.0, qk_norm=True, window=1024, seg_len=(64, 768), seed=1004),
+    Workload("sssl_short_gqa8x4_T2048_D96_rope_qknorm_win1024", B=16, T=2048, Hq=8, Hkv=4, D=96,
+             rope_base=10000.0, qk_norm=True, window=1024, seed=1005),
 ]
 
 BY_NAME = {w.name: w for w in WORKLOADS}
