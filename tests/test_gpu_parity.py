@@ -3,7 +3,7 @@
 Tolerances (stated for the bf16 path): O relative L2 <= 1e-2 and max-abs <= 2e-2;
 dQ, dK, dV relative L2 <= 2e-2 each; LSE max-abs <= 1e-2 (internal).
 Small shapes cover every option, ragged tails (T not a multiple of the 128-row tile),
-T = 1, odd group sizes and windows that bind.  The five named workloads run at full size
+T = 1, odd group sizes and windows that bind.  The named workloads run at full size
 in the launch configuration the benchmark times, checked against the oracle on sampled
 batch rows (batch rows are independent, so a row's outputs and gradients are exact
 oracle targets).
