@@ -64,6 +64,7 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [pp, dp, dp, dp, dp, ip, dp, dp, dp]
         lib.oracle_qk_prologue.argtypes = [pp, ctypes.c_int, dp, ip, dp]
         lib.oracle_attn_probs.argtypes = [pp, dp, dp, ip, ctypes.c_int, ctypes.c_int, dp]
+        lib.oracle_attn_fwd_cached.argtypes = [pp, ctypes.c_int, dp, dp, dp, dp, dp]
         lib.oracle_segments.argtypes = [ctypes.c_int, ctypes.c_int, ip, ip, ip]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -136,6 +137,25 @@ def attn_bwd(q, k, v, dout, *, causal=True, window=0, softcap=0.0, rope_base=0.0
     if rc:
         raise ValueError("oracle_attn_bwd rejected its arguments")
     return dq, dk, dv
+
+
+def attn_fwd_cached(q, k_cache, v_cache, *, causal=True, window=0, softcap=0.0, rope_base=0.0,
+                    qk_norm=False, qk_norm_eps=1e-6, scale=0.0):
+    """Tq new (raw) queries over a cache of Tk keys (already normalised and rotated, as the
+    prologue stores them) and values: O [B,Tq,Hq,D], LSE [B,Hq,Tq], fp64.  Query i sits at
+    absolute position Tk - Tq + i."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Tq, Hq, D = q.shape
+    Tk, Hkv = kc.shape[1], kc.shape[2]
+    assert kc.shape == (B, Tk, Hkv, D) and vc.shape == kc.shape
+    p = _params(B, Tk, Hq, Hkv, D, causal, window, softcap, rope_base, qk_norm, qk_norm_eps, scale)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Tq), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_cached(ctypes.byref(p), int(Tq), _dptr(q), _dptr(kc), _dptr(vc), _dptr(o),
+                                        _dptr(lse))
+    if rc:
+        raise ValueError("oracle_attn_fwd_cached rejected its arguments")
+    return o, lse
 
 
 def qk_prologue(x, *, rope_base=0.0, qk_norm=False, qk_norm_eps=1e-6, segment_ids=None):

@@ -341,6 +341,61 @@ int oracle_attn_bwd(const oracle_params* p, const double* q, const double* k, co
     return 0;
 }
 
+/* Attention of Tq new queries over a key/value cache of p->T entries (KV-cache decoding):
+ * "Build and Train a MiniGPT with JAX", section "Bonus: KV Caching".  The new queries are
+ * the last Tq positions of the sequence: offset = T - Tq, and query i sits at absolute
+ * position offset + i, so it may see key j only when j <= offset + i (causal); with a
+ * window also offset + i - j < W.  The cache holds keys as they were stored after their own
+ * norm and RoPE (k'), and the values; the raw queries get the norm and RoPE here, at their
+ * absolute positions.  q, o [B,Tq,Hq,D]; kc, vc [B,T,Hkv,D]; lse [B,Hq,Tq]. */
+int oracle_attn_fwd_cached(const oracle_params* p, int Tq, const double* q, const double* kc,
+                           const double* vc, double* o, double* lse) {
+    if (check(p) || Tq < 0 || Tq > p->T) return 1;
+    const int B = p->B, T = p->T, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = p->Hq / p->Hkv;
+    const int offset = T - Tq;
+    const double sc = eff_scale(p);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            const int kvh = h / G;
+            double* qp = (double*)malloc(sizeof(double) * (size_t)D);
+            double* s = (double*)malloc(sizeof(double) * ((size_t)T + 1));
+            for (int i = 0; i < Tq; ++i) {
+                const int pos = offset + i;
+                norm_rope_vec(p, q + idx4(b, i, h, 0, Tq, Hq, D), pos, qp);
+                double m = -INFINITY;
+                for (int j = 0; j < T; ++j) {
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += qp[d] * kc[idx4(b, j, kvh, d, T, Hkv, D)];
+                    acc *= sc;
+                    if (p->softcap > 0.0) acc = p->softcap * tanh(acc / p->softcap);
+                    int vis = 1;
+                    if (p->causal && j > pos) vis = 0;
+                    if (p->window > 0) {
+                        const int dd = pos - j;
+                        if (dd >= p->window || (!p->causal && -dd >= p->window)) vis = 0;
+                    }
+                    s[j] = vis ? acc : -INFINITY;
+                    if (s[j] > m) m = s[j];
+                }
+                double l = 0.0;
+                for (int j = 0; j < T; ++j) {
+                    s[j] = (s[j] == -INFINITY) ? 0.0 : exp(s[j] - m);
+                    l += s[j];
+                }
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j < T; ++j) acc += s[j] * vc[idx4(b, j, kvh, d, T, Hkv, D)];
+                    o[idx4(b, i, h, d, Tq, Hq, D)] = acc / l;
+                }
+                lse[((size_t)b * Hq + h) * Tq + i] = m + log(l);
+            }
+            free(qp);
+            free(s);
+        }
+    return 0;
+}
+
 /* Thread control for the CPU-baseline timing (OpenMP over (b, h) units). */
 #ifdef _OPENMP
 #include <omp.h>
