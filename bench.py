@@ -38,7 +38,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from causal_self_attention_gqa_b200.workloads import BY_NAME, WORKLOADS, make_inputs  # noqa: E402
+from causal_self_attention_gqa_b200.workloads import (BY_NAME, DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
+                                                      make_decode_inputs, make_inputs)
 
 DEFAULT_WORKLOAD = WORKLOADS[3].name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -284,6 +285,62 @@ def profile_step(w):
     return 0 if rc == 0 else 1
 
 
+def run_decode(args):
+    """KV-cache decoding (csa_attn_decode), 1 GPU: cache bytes read per second against the
+    measured HBM copy bandwidth.  The K/V cache (201 MB at the default shape) is larger than
+    L2, so every step streams it from HBM; no flush is needed between steps."""
+    from causal_self_attention_gqa_b200 import _binding as csa
+    w = DECODE_WORKLOADS[0]
+    if args.batch > 0:
+        w = w.with_(B=args.batch)
+    dev = torch.device("cuda:0")
+    inp = make_decode_inputs(w)
+    q, kc, vc = (inp[n].to(dev) for n in ("q", "k_cache", "v_cache"))
+    kw = w.options()
+    p = csa.make_params(w.B, w.Tk, w.Hq, w.Hkv, w.D, **kw)
+    ws = torch.empty(csa.decode_workspace_size(p, w.Tq), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        csa.attn_decode(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {csa.status_string(rc)}")
+    csa.timing_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        csa.attn_decode(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    csa.timing_enable(False)
+    kt = csa.timing_collect()
+    ms = e0.elapsed_time(e1) / args.steps
+    cache_bytes = 2 * w.B * w.Tk * w.Hkv * w.D * 2
+    io_bytes = cache_bytes + 2 * q.numel() * 2 + lse.numel() * 4
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    split_ms = kt["k_decode_split"][0] / max(kt["k_decode_split"][1], 1)
+    gbs = io_bytes / (ms * 1e-3) / 1e9
+    split_gbs = cache_bytes / (split_ms * 1e-3) / 1e9
+    line = {
+        "metric": "KV-cache decode step: bytes read per second (cache + queries + outputs)", "value": gbs,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "Tk": w.Tk, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "options": kw, "l2": "cache larger than L2, streamed every step"},
+        "tokens_per_s": w.B * w.Tq / (ms * 1e-3),
+        "kernels": {n: {"ms_avg": t / c if c else 0.0, "launches": c} for n, (t, c) in kt.items() if c},
+        "roofline": {"bound": "hbm", "achieved": split_gbs, "peak": hbm, "unit": "GB/s", "frac": split_gbs / hbm,
+                     "traffic": None, "kernel": "k_decode_split", "peak_source": f"{src}, hbm_gbs"},
+        "gpu_launches": sum(c for _, c in kt.values()),
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -294,6 +351,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end leg (default: min(K, 20))")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling cases)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the KV-cache decode step (csa_attn_decode) instead of the training step")
     ap.add_argument("--profile-step", action="store_true",
                     help="one warm-up step and one plain step, nothing else: a small case for ncu")
     args = ap.parse_args()
@@ -302,6 +361,8 @@ def main():
         w = w.with_(B=args.batch)
     if args.profile_step:
         return profile_step(w)
+    if args.decode:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -376,6 +437,7 @@ def main():
 
     # per-kernel times (library events on the launch stream, same timed region)
     launches = sum(c for _, c in kt.values())
+    kt = {name: tc for name, tc in kt.items() if tc[1] > 0}
     per_kernel = {name: {"ms_avg": (t / c if c else 0.0), "launches": c, "share": 0.0} for name, (t, c) in kt.items()}
     tot_k = sum(t for t, _ in kt.values()) or 1.0
     for name, (t, c) in kt.items():

@@ -25,6 +25,12 @@ cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMa
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
                        const float* lse, const float* delta, float* dq_acc, cudaStream_t st);
+DecodePlan decode_plan(const Problem& P, int Tq);
+cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q, float* qs, cudaStream_t st);
+cudaError_t launch_decode_split(const Problem& P, const DecodePlan& d, const float* qs, const void* kc,
+                                const void* vc, float* part, cudaStream_t st);
+cudaError_t launch_decode_combine(const Problem& P, const DecodePlan& d, const float* part, void* o, float* lse,
+                                  cudaStream_t st);
 
 int num_sms() {
     static int cache[64] = {0};
@@ -238,6 +244,7 @@ Problem make_problem(const csa_params& p, int* status) {
     P.cap_in = P.softcap > 0.f ? (float)((double)P.scale / (double)P.softcap) : 0.f;
     P.cap_log2 = (float)((double)P.softcap * 1.4426950408889634);
     P.rope = p.rope_base > 0.f ? 1 : 0;
+    P.rope_log_base = p.rope_base > 0.f ? log((double)p.rope_base) : 0.0;
     P.qk_norm = p.qk_norm;
     P.eps = p.qk_norm_eps;
     P.seg_start = nullptr;
@@ -247,7 +254,7 @@ Problem make_problem(const csa_params& p, int* status) {
     P.div_hkv = make_fastdiv((uint32_t)p.Hkv);
     P.div_t = make_fastdiv((uint32_t)(p.T > 0 ? p.T : 1));
     P.status = status;
-    P.counters = status + 1;
+    P.counters = status ? status + 1 : nullptr;
     return P;
 }
 
@@ -392,6 +399,55 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
     return attn_bwd(p, q, k, v, o, dout, lse, segment_ids, dq, dk, dv, workspace, workspace_bytes, stream, true);
 }
 
+// ------------------------------------------------------------------ KV-cache decode
+// Tq new queries over a cache of p->T entries; the rows of one (b, kv head), G * Tq, are at
+// most 16 (the decode kernel keeps them in registers).
+static int check_decode(const csa_params* p, int Tq) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (Tq < 1 || Tq > 16 || Tq > p->T) return CSA_ERR_INVALID_ARG;
+    if ((p->Hq / p->Hkv) * Tq > 16) return CSA_ERR_NOT_IMPLEMENTED;
+    return CSA_OK;
+}
+
+static size_t decode_ws_bytes(const csa_params* p, int Tq) {
+    const Problem P = make_problem(*p, nullptr);
+    const DecodePlan d = decode_plan(P, Tq);
+    return kAlign + up(d.qs_bytes) + up(d.part_bytes);
+}
+
+size_t csa_decode_workspace_size(const csa_params* p, int Tq) {
+    if (check_decode(p, Tq) != CSA_OK) return 0;
+    return decode_ws_bytes(p, Tq);
+}
+
+int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_cache, const void* v_cache, void* o,
+                    float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_decode(p, Tq);
+    if (rc) return rc;
+    if (p->B == 0) return CSA_OK;
+    if (!q || !k_cache || !v_cache || !o || !lse || !workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(workspace, 256))
+        return CSA_ERR_ALIGNMENT;
+    if (workspace_bytes < decode_ws_bytes(p, Tq)) return CSA_ERR_WORKSPACE;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    if (cudaMemsetAsync(w, 0, 4 * sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    const Problem P = make_problem(*p, reinterpret_cast<int*>(w));
+    const DecodePlan d = decode_plan(P, Tq);
+    float* qs = reinterpret_cast<float*>(w + kAlign);
+    float* part = reinterpret_cast<float*>(w + kAlign + up(d.qs_bytes));
+    if ((rc = timed(kDecodeQ, st, [&] { return launch_decode_q(P, d, q, qs, st); }))) return rc;
+    if ((rc = timed(kDecodeSplit, st, [&] { return launch_decode_split(P, d, qs, k_cache, v_cache, part, st); })))
+        return rc;
+    return timed(kDecodeCombine, st, [&] { return launch_decode_combine(P, d, part, o, lse, st); });
+}
+
 int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace) return CSA_ERR_INVALID_ARG;
     if (!aligned(workspace, 256)) return CSA_ERR_ALIGNMENT;
@@ -468,8 +524,9 @@ int csa_timing_collect(double* total_ms, int* launches, int n) {
 int csa_num_kernels(void) { return kNumKernels; }
 
 const char* csa_kernel_name(int k) {
-    static const char* names[kNumKernels] = {"k_prep", "k_qk_prologue", "k_attn_fwd",
-                                             "k_bwd_pre", "k_attn_bwd", "k_grad_finalize"};
+    static const char* names[kNumKernels] = {"k_prep",          "k_qk_prologue", "k_attn_fwd",
+                                             "k_bwd_pre",       "k_attn_bwd",    "k_grad_finalize",
+                                             "k_decode_q",      "k_decode_split", "k_decode_combine"};
     return (k >= 0 && k < kNumKernels) ? names[k] : "";
 }
 

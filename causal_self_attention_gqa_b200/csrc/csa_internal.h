@@ -49,16 +49,26 @@ struct Problem {
     const int32_t* seg_start;  // [B, T] first index of each token's segment, or null
     const int32_t* seg_end;    // [B, T] one past its last index, or null
     const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
+    double rope_log_base;      // ln(base) when RoPE is on
     FastDiv div_hq, div_hkv, div_t;  // row -> (token, head), token -> (batch row, position)
     int* status;               // device status word (workspace, or the caller's)
     int* counters;             // [2] work-item counters of the persistent kernels (workspace,
                                // zeroed by every call): forward, backward
 };
 
+// Work split of the KV-cache decode (decode.cu): Tq new queries, R = G * Tq rows per
+// (b, kv head), the cache cut into `splits` ranges of keys_per_split keys.
+struct DecodePlan {
+    int Tq, R, splits, keys_per_split;
+    size_t qs_bytes, part_bytes;
+};
+
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 
 // Kernel ids for the timing interface (order = csa_kernel_name()).
-enum KernelId { kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kNumKernels };
+enum KernelId {
+    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecodeQ, kDecodeSplit, kDecodeCombine, kNumKernels
+};
 
 }  // namespace csa

@@ -101,3 +101,49 @@ def make_inputs(w: Workload, *, need_grad_input: bool = True) -> dict:
         lo, hi = w.seg_len
         out["segment_ids"] = torch.from_numpy(packed_segment_ids(w.B, w.T, lo, hi, w.seed))
     return out
+
+
+# KV-cache decoding: B rows of Tq new raw queries over a cache of Tk entries.  The cached keys
+# stand for keys already passed through the norm and RoPE: unit-RMS N(0,1) draws, like the
+# normalised keys of the QK-norm models.
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Tk: int
+    Tq: int
+    Hq: int
+    Hkv: int
+    D: int
+    causal: bool = True
+    window: int = 0
+    softcap: float = 0.0
+    rope_base: float = 0.0
+    qk_norm: bool = False
+    qk_norm_eps: float = 1e-6
+    scale: float = 0.0
+    seed: int = 0
+
+    def options(self) -> dict:
+        return dict(causal=self.causal, window=self.window, softcap=self.softcap, rope_base=self.rope_base,
+                    qk_norm=self.qk_norm, qk_norm_eps=self.qk_norm_eps, scale=self.scale)
+
+    def with_(self, **kw) -> "DecodeWorkload":
+        return replace(self, **kw)
+
+
+# One decoding step of the 181M model on a batch of 16 sequences with 8192 tokens of history.
+DECODE_WORKLOADS = [
+    DecodeWorkload("decode_gpt181m_gqa8x4_D96_rope_qknorm_cache8192", B=16, Tk=8192, Tq=1, Hq=8, Hkv=4, D=96,
+                   rope_base=10000.0, qk_norm=True, seed=2000),
+]
+
+
+def make_decode_inputs(w: DecodeWorkload) -> dict:
+    """bf16 CPU tensors q [B,Tq,Hq,D] (raw), k_cache / v_cache [B,Tk,Hkv,D]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    q = torch.randn((w.B, w.Tq, w.Hq, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return dict(q=q, k_cache=kc, v_cache=vc)

@@ -112,6 +112,26 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
                            const int32_t* segment_ids, void* dq, void* dk, void* dv,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* KV-cache decoding ("Build and Train a MiniGPT with JAX", section "Bonus: KV Caching"):
+ * Tq new queries attend over a cache of p->T entries.  With offset = p->T - Tq, query i sits
+ * at absolute position offset + i and sees cache entry j when j <= offset + i (p->causal = 1;
+ * 0: every entry) and, with a window W > 0, when |offset + i - j| < W.
+ *   q        [B, Tq, Hq, D] bf16, raw: QK-norm and RoPE (at the absolute positions) are applied
+ *            here when p->qk_norm / p->rope_base ask for them;
+ *   k_cache  [B, p->T, Hkv, D] bf16, keys as stored after their own QK-norm and RoPE (the
+ *            forward's prologue output for the same positions);
+ *   v_cache  [B, p->T, Hkv, D] bf16;
+ *   o        [B, Tq, Hq, D] bf16;  lse [B, Hq, Tq] fp32 (natural log).
+ * 1 <= Tq <= min(16, p->T) (CSA_ERR_INVALID_ARG otherwise) and (Hq / Hkv) * Tq <= 16
+ * (CSA_ERR_NOT_IMPLEMENTED otherwise); segment_ids do not apply.  Tensors 16-byte aligned,
+ * workspace 256-byte aligned and at least csa_decode_workspace_size(p, Tq) bytes (0 when the
+ * arguments are invalid).  The pages give no kernel for this; it is memory-bound and runs on
+ * the CUDA cores, split over the cache, then merged. */
+size_t csa_decode_workspace_size(const csa_params* p, int Tq);
+int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_cache,
+                    const void* v_cache, void* o, float* lse, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last call that used it (CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA when the
  * synchronisation itself failed).  Resets the recorded status to CSA_OK. */

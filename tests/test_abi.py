@@ -102,4 +102,23 @@ def test_status_strings(b):
         assert b.status_string(code)
     assert b.status_string(6) == "a bounded wait inside a kernel ran out"
     assert b.kernel_names() == ["k_prep", "k_qk_prologue", "k_attn_fwd", "k_bwd_pre", "k_attn_bwd",
-                                "k_grad_finalize"]
+                                "k_grad_finalize", "k_decode_q", "k_decode_split", "k_decode_combine"]
+
+
+def test_decode_arguments_are_checked_on_the_host(b):
+    """csa_attn_decode: Tq range, rows per KV head, alignment and workspace size are
+    rejected before anything is enqueued (fake pointers: every call here fails a check)."""
+    p = b.make_params(2, 64, 8, 4, 96, rope_base=10000.0, qk_norm=True)
+    assert b.decode_workspace_size(p, 1) > 0
+    assert b.decode_workspace_size(p, 0) == 0          # Tq < 1
+    assert b.decode_workspace_size(p, 17) == 0         # Tq > 16
+    assert b.decode_workspace_size(b.make_params(2, 4, 8, 4, 96), 5) == 0   # Tq > cache length
+    assert b.decode_workspace_size(b.make_params(2, 64, 32, 1, 64), 1) == 0  # 32 rows per KV head
+    dec = b.lib.csa_attn_decode
+    ptr = [0x1000 * (i + 1) for i in range(6)]
+    assert dec(ctypes.byref(p), 0, *ptr[:5], 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
+    assert dec(ctypes.byref(b.make_params(2, 64, 32, 1, 64)), 1, *ptr[:5], 0x10000, 1 << 30,
+               None) == b.CSA_ERR_NOT_IMPLEMENTED
+    assert dec(ctypes.byref(p), 1, 0x1008, *ptr[1:5], 0x10000, 1 << 30, None) == b.CSA_ERR_ALIGNMENT
+    assert dec(ctypes.byref(p), 1, *ptr[:5], 0x10000, 64, None) == b.CSA_ERR_WORKSPACE
+    assert dec(ctypes.byref(p), 1, None, *ptr[1:5], 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
