@@ -11,11 +11,12 @@
 // Decoding reads the whole cache for a handful of queries, so it is bound by HBM bandwidth,
 // not by the tensor cores: the work runs on the CUDA cores, split over the cache.
 //   k_decode_q       q' = RoPE(RMSNorm(q)) * scale for the G * Tq rows of every (b, kv head),
-//                    fp32, cos/sin from fp64 (positions reach 2^20)
+//                    fp32; the rotation phase is formed and reduced in fp64 (positions reach
+//                    2^20)
 //   k_decode_split   one CTA per (key range, kv head, b): each warp streams 32 keys at a time
 //                    (lane = key for the scores, lane = 4 dimensions for P V), online softmax
-//                    in log2 units; the CTA's partial (m, l, o) goes to the workspace
-//   k_decode_combine merges the partials of all key ranges: o = sum 2^(m_s - m) o_s / l
+//                    in log2 units; the CTA's partial (m, l, o) goes to the workspace, and the
+//                    last CTA of each (b, kv head) merges them: o = sum 2^(m_s - m) o_s / l
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -60,11 +61,16 @@ __global__ void __launch_bounds__(128) k_decode_q(const __nv_bfloat16* __restric
 #pragma unroll
         for (int t = 0; t < kPer; ++t) {
             const int d = lane + 32 * t, d2 = d % (D / 2);
-            const double theta = exp((-2.0 * d2 / D) * (double)P.rope_log_base);
-            double s, c;
-            sincos((double)pos * theta, &s, &c);
+            // phase pos * theta in fp64 (it reaches ~1e6 rad), reduced to [-pi, pi] with a
+            // two-part 2 pi (Cody-Waite), then the fp32 sine / cosine of the remainder
+            const double theta = exp((-2.0 * d2 / D) * P.rope_log_base);
+            const double phi = (double)pos * theta;
+            const double k = rint(phi * 0.15915494309189535);  // 1 / (2 pi)
+            const double red = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, phi));
+            float sn, cs;
+            sincosf((float)red, &sn, &cs);
             const float a = y[d2], bb = y[d2 + D / 2];
-            out[t] = (d < D / 2) ? a * (float)c - bb * (float)s : bb * (float)c + a * (float)s;
+            out[t] = (d < D / 2) ? a * cs - bb * sn : bb * cs + a * sn;
         }
         __syncwarp();
 #pragma unroll
@@ -85,7 +91,37 @@ struct DecArgs {
     const __nv_bfloat16* kc;       // [B, Tk, Hkv, D]
     const __nv_bfloat16* vc;       // [B, Tk, Hkv, D]
     float* part;                   // [B, Hkv, splits, R, D + 2]: o (unnormalised), m, l
+    int* done;                     // [B, Hkv] key ranges finished (zeroed by the call)
+    __nv_bfloat16* o;              // [B, Tq, Hq, D]
+    float* lse;                    // [B, Hq, Tq]
 };
+
+// o and LSE of one (b, kv head) from the partials of all its key ranges:
+// m = max_s m_s, l = sum_s 2^(m_s - m) l_s, o = sum_s 2^(m_s - m) o_s / l.  The partials come
+// from other CTAs: read through L2 (ld.global.cg), never from this SM's L1.
+template <int D>
+__device__ void merge_partials(const DecArgs& A, int b, int kvh) {
+    const Problem& P = A.P;
+    const float* src = A.part + (((size_t)b * P.Hkv + kvh) * A.splits) * A.R * (D + 2);
+    for (int e = threadIdx.x; e < A.R * D; e += blockDim.x) {
+        const int r = e / D, d = e % D;
+        float mm = -INFINITY;
+        for (int s = 0; s < A.splits; ++s) mm = fmaxf(mm, __ldcg(src + ((size_t)s * A.R + r) * (D + 2) + D));
+        float acc = 0.f, ll = 0.f;
+        for (int s = 0; s < A.splits; ++s) {
+            const float* ps = src + ((size_t)s * A.R + r) * (D + 2);
+            const float ms = __ldcg(ps + D);
+            const float f = (ms == -INFINITY) ? 0.f : ex2(ms - mm);
+            acc += f * __ldcg(ps + d);
+            ll += f * __ldcg(ps + D + 1);
+        }
+        const int i = r % A.Tq, h = kvh * P.G + r / A.Tq;
+        A.o[((size_t)(b * A.Tq + i) * P.Hq + h) * D + d] = __float2bfloat16_rn(ll > 0.f ? acc / ll : 0.f);
+        if (d == 0)
+            A.lse[((size_t)b * P.Hq + h) * A.Tq + i] =
+                (ll > 0.f) ? (mm + __log2f(ll)) * 0.6931471805599453f : -INFINITY;
+    }
+}
 
 // Visible keys of row r (query i = r % Tq): [lo, hi].
 __device__ __forceinline__ void dec_bounds(const Problem& P, int Tq, int r, int& lo, int& hi) {
@@ -99,7 +135,7 @@ __device__ __forceinline__ void dec_bounds(const Problem& P, int Tq, int r, int&
 }
 
 template <int D, int RMAX, bool CAP>
-__global__ void __launch_bounds__(kDecThreads, 4) k_decode_split(const DecArgs A) {
+__global__ void __launch_bounds__(kDecThreads, RMAX >= 16 ? 2 : 4) k_decode_split(const DecArgs A) {
     const Problem& P = A.P;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -235,32 +271,16 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode_split(const DecArgs A
             dst[(size_t)r * (D + 2) + D + 1] = ll;
         }
     }
-}
-
-// ------------------------------------------------------------------ combine the key ranges
-// One CTA per (b, kv head); thread e covers (row, dimension) pairs.
-template <int D>
-__global__ void __launch_bounds__(128) k_decode_combine(const DecArgs A, __nv_bfloat16* __restrict__ o,
-                                                        float* __restrict__ lse) {
-    const Problem& P = A.P;
-    const int kvh = blockIdx.x % P.Hkv, b = blockIdx.x / P.Hkv;
-    const float* src = A.part + (((size_t)b * P.Hkv + kvh) * A.splits) * A.R * (D + 2);
-    for (int e = threadIdx.x; e < A.R * D; e += blockDim.x) {
-        const int r = e / D, d = e % D;
-        float mm = -INFINITY;
-        for (int s = 0; s < A.splits; ++s) mm = fmaxf(mm, src[((size_t)s * A.R + r) * (D + 2) + D]);
-        float acc = 0.f, ll = 0.f;
-        for (int s = 0; s < A.splits; ++s) {
-            const float* ps = src + ((size_t)s * A.R + r) * (D + 2);
-            const float f = (ps[D] == -INFINITY) ? 0.f : ex2(ps[D] - mm);
-            acc += f * ps[d];
-            ll += f * ps[D + 1];
-        }
-        const int i = r % A.Tq, h = kvh * P.G + r / A.Tq;
-        o[((size_t)(b * A.Tq + i) * P.Hq + h) * D + d] = __float2bfloat16_rn(ll > 0.f ? acc / ll : 0.f);
-        if (d == 0)
-            lse[((size_t)b * P.Hq + h) * A.Tq + i] = (ll > 0.f) ? (mm + __log2f(ll)) * 0.6931471805599453f : -INFINITY;
-    }
+    // the last CTA of this (b, kv head) to finish merges every key range (no waiting: the
+    // others have published their partials before counting themselves done)
+    __threadfence();
+    __syncthreads();
+    __shared__ int last;
+    if (threadIdx.x == 0) last = (atomicAdd(&A.done[b * P.Hkv + kvh], 1) == A.splits - 1) ? 1 : 0;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    merge_partials<D>(A, b, kvh);
 }
 
 // ------------------------------------------------------------------ host side
@@ -279,11 +299,12 @@ DecodePlan decode_plan(const Problem& P, int Tq) {
     d.splits = (P.T + d.keys_per_split - 1) / d.keys_per_split;
     d.qs_bytes = (size_t)P.B * P.Hkv * d.R * P.D * sizeof(float);
     d.part_bytes = (size_t)P.B * P.Hkv * d.splits * d.R * (P.D + 2) * sizeof(float);
+    d.done_bytes = (size_t)P.B * P.Hkv * sizeof(int);
     return d;
 }
 
 static DecArgs dec_args(const Problem& P, const DecodePlan& d, const float* qs, const void* kc, const void* vc,
-                        float* part) {
+                        float* part, int* done, void* o, float* lse) {
     DecArgs A;
     A.P = P;
     A.Tq = d.Tq;
@@ -294,6 +315,9 @@ static DecArgs dec_args(const Problem& P, const DecodePlan& d, const float* qs, 
     A.kc = static_cast<const __nv_bfloat16*>(kc);
     A.vc = static_cast<const __nv_bfloat16*>(vc);
     A.part = part;
+    A.done = done;
+    A.o = static_cast<__nv_bfloat16*>(o);
+    A.lse = lse;
     return A;
 }
 
@@ -331,18 +355,9 @@ cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q
 }
 
 cudaError_t launch_decode_split(const Problem& P, const DecodePlan& d, const float* qs, const void* kc,
-                                const void* vc, float* part, cudaStream_t st) {
-    const DecArgs A = dec_args(P, d, qs, kc, vc, part);
+                                const void* vc, float* part, int* done, void* o, float* lse, cudaStream_t st) {
+    const DecArgs A = dec_args(P, d, qs, kc, vc, part, done, o, lse);
 #define CALL(D_) ((P.softcap > 0.f) ? launch_split_r<D_, true>(A, st) : launch_split_r<D_, false>(A, st))
-    CSA_DEC_DISPATCH(CALL)
-#undef CALL
-}
-
-cudaError_t launch_decode_combine(const Problem& P, const DecodePlan& d, const float* part, void* o, float* lse,
-                                  cudaStream_t st) {
-    const DecArgs A = dec_args(P, d, nullptr, nullptr, nullptr, const_cast<float*>(part));
-#define CALL(D_)                                                                                          \
-    (k_decode_combine<D_><<<P.B * P.Hkv, 128, 0, st>>>(A, static_cast<__nv_bfloat16*>(o), lse), cudaGetLastError())
     CSA_DEC_DISPATCH(CALL)
 #undef CALL
 }
