@@ -28,9 +28,7 @@ cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMa
 DecodePlan decode_plan(const Problem& P, int Tq);
 cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q, float* qs, cudaStream_t st);
 cudaError_t launch_decode_split(const Problem& P, const DecodePlan& d, const float* qs, const void* kc,
-                                const void* vc, float* part, cudaStream_t st);
-cudaError_t launch_decode_combine(const Problem& P, const DecodePlan& d, const float* part, void* o, float* lse,
-                                  cudaStream_t st);
+                                const void* vc, float* part, int* done, void* o, float* lse, cudaStream_t st);
 
 int num_sms() {
     static int cache[64] = {0};
@@ -413,7 +411,7 @@ static int check_decode(const csa_params* p, int Tq) {
 static size_t decode_ws_bytes(const csa_params* p, int Tq) {
     const Problem P = make_problem(*p, nullptr);
     const DecodePlan d = decode_plan(P, Tq);
-    return kAlign + up(d.qs_bytes) + up(d.part_bytes);
+    return kAlign + up(d.qs_bytes) + up(d.part_bytes) + up(d.done_bytes);
 }
 
 size_t csa_decode_workspace_size(const csa_params* p, int Tq) {
@@ -442,10 +440,14 @@ int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_ca
     const DecodePlan d = decode_plan(P, Tq);
     float* qs = reinterpret_cast<float*>(w + kAlign);
     float* part = reinterpret_cast<float*>(w + kAlign + up(d.qs_bytes));
+    int* done = reinterpret_cast<int*>(w + kAlign + up(d.qs_bytes) + up(d.part_bytes));
+    if (cudaMemsetAsync(done, 0, d.done_bytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
     if ((rc = timed(kDecodeQ, st, [&] { return launch_decode_q(P, d, q, qs, st); }))) return rc;
-    if ((rc = timed(kDecodeSplit, st, [&] { return launch_decode_split(P, d, qs, k_cache, v_cache, part, st); })))
-        return rc;
-    return timed(kDecodeCombine, st, [&] { return launch_decode_combine(P, d, part, o, lse, st); });
+    return timed(kDecodeSplit, st,
+                 [&] { return launch_decode_split(P, d, qs, k_cache, v_cache, part, done, o, lse, st); });
 }
 
 int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
@@ -526,7 +528,7 @@ int csa_num_kernels(void) { return kNumKernels; }
 const char* csa_kernel_name(int k) {
     static const char* names[kNumKernels] = {"k_prep",          "k_qk_prologue", "k_attn_fwd",
                                              "k_bwd_pre",       "k_attn_bwd",    "k_grad_finalize",
-                                             "k_decode_q",      "k_decode_split", "k_decode_combine"};
+                                             "k_decode_q",      "k_decode_split"};
     return (k >= 0 && k < kNumKernels) ? names[k] : "";
 }
 

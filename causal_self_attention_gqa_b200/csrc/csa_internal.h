@@ -60,7 +60,7 @@ struct Problem {
 // (b, kv head), the cache cut into `splits` ranges of keys_per_split keys.
 struct DecodePlan {
     int Tq, R, splits, keys_per_split;
-    size_t qs_bytes, part_bytes;
+    size_t qs_bytes, part_bytes, done_bytes;
 };
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -68,7 +68,7 @@ int num_sms();
 
 // Kernel ids for the timing interface (order = csa_kernel_name()).
 enum KernelId {
-    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecodeQ, kDecodeSplit, kDecodeCombine, kNumKernels
+    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecodeQ, kDecodeSplit, kNumKernels
 };
 
 }  // namespace csa

@@ -102,7 +102,7 @@ def test_status_strings(b):
         assert b.status_string(code)
     assert b.status_string(6) == "a bounded wait inside a kernel ran out"
     assert b.kernel_names() == ["k_prep", "k_qk_prologue", "k_attn_fwd", "k_bwd_pre", "k_attn_bwd",
-                                "k_grad_finalize", "k_decode_q", "k_decode_split", "k_decode_combine"]
+                                "k_grad_finalize", "k_decode_q", "k_decode_split"]
 
 
 def test_decode_arguments_are_checked_on_the_host(b):
