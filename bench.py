@@ -341,6 +341,66 @@ def run_decode(args):
     return 0
 
 
+def run_prefill(args):
+    """Forward over a KV cache (csa_attn_prefill): a 2048-token chunk at the end of an
+    8192-entry cache, 181M shape, batch 4; algorithmic TFLOP/s (4 D per visible pair and query
+    head) against the measured bf16 peak.  The caches (101 MB) and queries exceed L2 together."""
+    from causal_self_attention_gqa_b200 import _binding as csa
+    from causal_self_attention_gqa_b200.workloads import DecodeWorkload
+    w = DecodeWorkload("prefill_gpt181m_gqa8x4_D96_rope_qknorm_chunk2048_cache8192", B=args.batch or 4, Tk=8192,
+                       Tq=2048, Hq=8, Hkv=4, D=96, rope_base=10000.0, qk_norm=True, seed=2001)
+    dev = torch.device("cuda:0")
+    inp = make_decode_inputs(w)
+    q, kc, vc = (inp[n].to(dev) for n in ("q", "k_cache", "v_cache"))
+    kw = w.options()
+    p = csa.make_params(w.B, w.Tk, w.Hq, w.Hkv, w.D, **kw)
+    ws = torch.empty(csa.prefill_workspace_size(p, w.Tq), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        csa.attn_prefill(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {csa.status_string(rc)}")
+    csa.timing_enable(True)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        csa.attn_prefill(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    csa.timing_enable(False)
+    kt = {n: tc for n, tc in csa.timing_collect().items() if tc[1] > 0}
+    ms = sum(a.elapsed_time(b) for a, b in times) / args.steps
+    off = w.Tk - w.Tq
+    pairs = sum(off + i + 1 for i in range(w.Tq))  # causal, per (b, query head)
+    flops = 4.0 * w.D * w.Hq * w.B * pairs
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fwd_ms = kt["k_attn_fwd"][0] / kt["k_attn_fwd"][1]
+    line = {
+        "metric": "forward over a KV cache (chunked prefill): algorithmic TFLOP/s", "value": flops / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "Tk": w.Tk, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "options": kw, "l2": "flushed between timed steps (256 MiB write, outside the events)"},
+        "tokens_per_s": w.B * w.Tq / (ms * 1e-3),
+        "kernels": {n: {"ms_avg": t / c, "launches": c} for n, (t, c) in kt.items()},
+        "roofline": {"bound": "tensor", "achieved": flops / (fwd_ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                     "frac": flops / (fwd_ms * 1e-3) / 1e12 / peak, "traffic": None, "kernel": "k_attn_fwd",
+                     "peak_source": f"{src}, bf16_tflops"},
+        "gpu_launches": sum(c for _, c in kt.values()),
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -351,6 +411,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end leg (default: min(K, 20))")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling cases)")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the forward over a KV cache (csa_attn_prefill) instead of the training step")
     ap.add_argument("--decode", action="store_true",
                     help="time the KV-cache decode step (csa_attn_decode) instead of the training step")
     ap.add_argument("--profile-step", action="store_true",
@@ -363,6 +425,8 @@ def main():
         return profile_step(w)
     if args.decode:
         return run_decode(args)
+    if args.prefill:
+        return run_prefill(args)
     if args.impl == "reference":
         return run_reference(args, w)
 

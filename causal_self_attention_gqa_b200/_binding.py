@@ -32,7 +32,8 @@ CSA_ERR_NOT_IMPLEMENTED = 8
 EXPORTED = ["csa_workspace_size", "csa_attn_fwd", "csa_attn_bwd", "csa_device_status",
             "csa_status_string", "csa_timing_enable", "csa_timing_collect", "csa_num_kernels",
             "csa_kernel_name", "csa_attn_fwd_static_scratch", "csa_selftest_bounded_wait",
-            "csa_attn_bwd_after_fwd", "csa_decode_workspace_size", "csa_attn_decode"]
+            "csa_attn_bwd_after_fwd", "csa_decode_workspace_size", "csa_attn_decode",
+            "csa_prefill_workspace_size", "csa_attn_prefill"]
 
 
 class Params(ctypes.Structure):
@@ -54,6 +55,11 @@ _lib.csa_attn_bwd.restype = ctypes.c_int
 _lib.csa_attn_bwd_after_fwd.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _vp, ctypes.c_size_t, _vp]
 _lib.csa_attn_bwd_after_fwd.restype = ctypes.c_int
+_lib.csa_prefill_workspace_size.argtypes = [ctypes.POINTER(Params), ctypes.c_int]
+_lib.csa_prefill_workspace_size.restype = ctypes.c_size_t
+_lib.csa_attn_prefill.argtypes = [ctypes.POINTER(Params), ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                  _vp]
+_lib.csa_attn_prefill.restype = ctypes.c_int
 _lib.csa_decode_workspace_size.argtypes = [ctypes.POINTER(Params), ctypes.c_int]
 _lib.csa_decode_workspace_size.restype = ctypes.c_size_t
 _lib.csa_attn_decode.argtypes = [ctypes.POINTER(Params), ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
@@ -191,6 +197,36 @@ def attn_bwd(q, k, v, o, do, lse, *, causal=True, window=0, softcap=0.0, rope_ba
     if rc != CSA_OK:
         raise CsaError(rc, "csa_attn_bwd_after_fwd" if after_fwd else "csa_attn_bwd")
     return dq, dk, dv
+
+
+def prefill_workspace_size(p: Params, Tq: int) -> int:
+    """csa_prefill_workspace_size: bytes of workspace csa_attn_prefill needs (0: invalid)."""
+    return int(_lib.csa_prefill_workspace_size(ctypes.byref(p), int(Tq)))
+
+
+def attn_prefill(q, k_cache, v_cache, *, causal=True, window=0, softcap=0.0, rope_base=0.0, qk_norm=False,
+                 qk_norm_eps=1e-6, scale=0.0, out=None, lse=None, workspace=None, stream=None):
+    """csa_attn_prefill: the forward of Tq new raw queries (the last Tq positions) over a cache
+    of Tk keys (stored after their own norm and RoPE) and values; o bf16, lse fp32."""
+    B, Tq, Hq, D = q.shape
+    Tk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _check_bf16("q", q, (B, Tq, Hq, D))
+    _check_bf16("k_cache", k_cache, (B, Tk, Hkv, D))
+    _check_bf16("v_cache", v_cache, (B, Tk, Hkv, D))
+    p = make_params(B, Tk, Hq, Hkv, D, causal=causal, window=window, softcap=softcap, rope_base=rope_base,
+                    qk_norm=qk_norm, qk_norm_eps=qk_norm_eps, scale=scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        n = prefill_workspace_size(p, Tq)
+        if n == 0:
+            raise CsaError(CSA_ERR_INVALID_ARG, "csa_prefill_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    rc = _lib.csa_attn_prefill(ctypes.byref(p), int(Tq), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != CSA_OK:
+        raise CsaError(rc, "csa_attn_prefill")
+    return o, lse
 
 
 def decode_workspace_size(p: Params, Tq: int) -> int:

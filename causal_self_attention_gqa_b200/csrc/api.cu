@@ -251,6 +251,9 @@ Problem make_problem(const csa_params& p, int* status) {
     P.div_hq = make_fastdiv((uint32_t)p.Hq);
     P.div_hkv = make_fastdiv((uint32_t)p.Hkv);
     P.div_t = make_fastdiv((uint32_t)(p.T > 0 ? p.T : 1));
+    P.Tq = p.T;
+    P.qoff = 0;
+    P.div_tq = P.div_t;
     P.status = status;
     P.counters = status ? status + 1 : nullptr;
     return P;
@@ -395,6 +398,71 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
                            const void* dout, const float* lse, const int32_t* segment_ids, void* dq, void* dk,
                            void* dv, void* workspace, size_t workspace_bytes, void* stream) {
     return attn_bwd(p, q, k, v, o, dout, lse, segment_ids, dq, dk, dv, workspace, workspace_bytes, stream, true);
+}
+
+// ------------------------------------------------------------------ forward over a KV cache
+// Tq queries at absolute positions T - Tq + i over a cache of p->T entries (chunked prefill);
+// the tensor-core forward with its own query length and offset.  Workspace: status slot,
+// RoPE table (positions 0..T-1), q' (queries only: the cache holds processed keys).
+static int check_prefill(const csa_params* p, int Tq) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (Tq < 1 || Tq > p->T) return CSA_ERR_INVALID_ARG;
+    return CSA_OK;
+}
+
+static size_t prefill_ws_bytes(const csa_params* p, int Tq, size_t* rope_off, size_t* qp_off) {
+    size_t off = kAlign;
+    *rope_off = off;
+    if (p->rope_base > 0.f) off += up((size_t)p->T * (p->D / 2) * 8);
+    *qp_off = off;
+    if (needs_prologue(*p)) off += up((size_t)p->B * Tq * p->Hq * p->D * 2);
+    return off;
+}
+
+size_t csa_prefill_workspace_size(const csa_params* p, int Tq) {
+    if (check_prefill(p, Tq) != CSA_OK) return 0;
+    size_t a, b;
+    return prefill_ws_bytes(p, Tq, &a, &b);
+}
+
+int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_cache, const void* v_cache, void* o,
+                     float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_prefill(p, Tq);
+    if (rc) return rc;
+    if (p->B == 0) return CSA_OK;
+    if (!q || !k_cache || !v_cache || !o || !lse || !workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(workspace, 256))
+        return CSA_ERR_ALIGNMENT;
+    size_t rope_off, qp_off;
+    if (workspace_bytes < prefill_ws_bytes(p, Tq, &rope_off, &qp_off)) return CSA_ERR_WORKSPACE;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    if (cudaMemsetAsync(w, 0, 4 * sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA_ERR_CUDA;
+    }
+    Problem P = make_problem(*p, reinterpret_cast<int*>(w));
+    P.Tq = Tq;
+    P.qoff = p->T - Tq;
+    P.div_tq = make_fastdiv((uint32_t)Tq);
+    float2* rope = p->rope_base > 0.f ? reinterpret_cast<float2*>(w + rope_off) : nullptr;
+    P.rope_cs = rope;
+    if (rope && (rc = timed(kPrep, st, [&] { return launch_prep(P, nullptr, nullptr, nullptr, rope, p->rope_base, st); })))
+        return rc;
+    const void* qq = q;
+    if (needs_prologue(*p)) {
+        void* qp = w + qp_off;
+        if ((rc = timed(kPrologue, st, [&] { return launch_prologue(P, q, nullptr, qp, nullptr, st); }))) return rc;
+        qq = qp;
+    }
+    CUtensorMap tq, tk, tv, to;
+    if (!make_map(&tq, qq, p->B, Tq, p->Hq, p->D) || !make_map(&tk, k_cache, p->B, p->T, p->Hkv, p->D) ||
+        !make_map(&tv, v_cache, p->B, p->T, p->Hkv, p->D) || !make_map(&to, o, p->B, Tq, p->Hq, p->D))
+        return CSA_ERR_CUDA;
+    return timed(kFwd, st, [&] { return launch_fwd(P, tq, tk, tv, to, lse, st); });
 }
 
 // ------------------------------------------------------------------ KV-cache decode

@@ -73,21 +73,22 @@ struct FwdArgs {
     int items;     // number of work items
 };
 
-// Keys visible to query row q: [lo, hi] (empty when lo > hi).
+// Keys visible to query row q (absolute position qoff + q): [lo, hi] (empty when lo > hi).
 __device__ __forceinline__ void row_bounds(const Problem& P, int b, int q, int& lo, int& hi) {
-    if (q >= P.T || q < 0) {
+    if (q >= P.Tq || q < 0) {
         lo = P.T;
         hi = -1;
         return;
     }
-    int l = 0, h = P.causal ? q : P.T - 1;
-    if (P.seg_start) {
+    const int pos = q + P.qoff;
+    int l = 0, h = P.causal ? min(pos, P.T - 1) : P.T - 1;
+    if (P.seg_start) {  // segments only without a cache (Tq = T, qoff = 0)
         l = P.seg_start[(size_t)b * P.T + q];
         h = min(h, P.seg_end[(size_t)b * P.T + q] - 1);
     }
     if (P.window > 0) {
-        l = max(l, q - P.window + 1);
-        if (!P.causal) h = min(h, q + P.window - 1);
+        l = max(l, pos - P.window + 1);
+        if (!P.causal) h = min(h, pos + P.window - 1);
     }
     lo = l;
     hi = h;
@@ -135,7 +136,7 @@ __device__ __forceinline__ FwdItem decode_item(const FwdArgs& A, int idx) {
     int lo0, hi0, lo1, hi1;
     row_bounds(P, w.b, w.mm[0] * kBM, lo0, hi0);
     const int last = w.two ? w.mm[1] : w.mm[0];
-    row_bounds(P, w.b, min(last * kBM + kBM - 1, P.T - 1), lo1, hi1);
+    row_bounds(P, w.b, min(last * kBM + kBM - 1, P.Tq - 1), lo1, hi1);
     w.kt_begin = lo0 / kBN;
     w.nkt = hi1 / kBN - w.kt_begin + 1;
     return w;
@@ -466,8 +467,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             tc_fence_before();
             warp_arrive(&o_empty[i]);
-            if (q < P.T)
-                A.lse[((size_t)w.b * P.Hq + h) * P.T + q] =
+            if (q < P.Tq)
+                A.lse[((size_t)w.b * P.Hq + h) * P.Tq + q] =
                     (l > 0.f) ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
             // O goes out through one shared staging tile (TMA box layout) and tiled TMA stores;
             // the two warpgroups take turns, warpgroup 0 first
@@ -524,7 +525,7 @@ static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.P = P;
     A.lse = lse;
     A.counter = P.counters;  // cleared together with the status word by the call
-    A.nqt = (P.T + kBM - 1) / kBM;
+    A.nqt = (P.Tq + kBM - 1) / kBM;
     if (P.G >= 2) {
         A.pairs = (P.G + 1) / 2;
         A.items = P.B * P.Hkv * A.pairs * A.nqt;

@@ -38,6 +38,10 @@ inline uint32_t fastdiv(uint32_t n, FastDiv f) {
 // Everything a kernel needs to know about the problem.
 struct Problem {
     int B, T, Hq, Hkv, D, G;
+    // Query rows and the absolute position of query row 0.  Tq = T and qoff = 0 everywhere
+    // except the forward over a key/value cache, where T is the cache length and the Tq
+    // queries are its last positions (qoff = T - Tq).
+    int Tq, qoff;
     int causal, window;
     float softcap;          // 0 = off
     float cap_in;           // scale / softcap: tanh argument per raw score (cap on)
@@ -50,7 +54,7 @@ struct Problem {
     const int32_t* seg_end;    // [B, T] one past its last index, or null
     const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
     double rope_log_base;      // ln(base) when RoPE is on
-    FastDiv div_hq, div_hkv, div_t;  // row -> (token, head), token -> (batch row, position)
+    FastDiv div_hq, div_hkv, div_t, div_tq;  // row -> (token, head), token -> (batch row, position)
     int* status;               // device status word (workspace, or the caller's)
     int* counters;             // [2] work-item counters of the persistent kernels (workspace,
                                // zeroed by every call): forward, backward

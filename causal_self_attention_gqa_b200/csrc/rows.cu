@@ -119,9 +119,9 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
     const uint32_t row = valid ? row_raw : 0;
     const bool is_q = row < rows_q;
     const uint32_t r = is_q ? row : row - rows_q;
-    const uint32_t tok = fastdiv(r, is_q ? P.div_hq : P.div_hkv);  // b * T + t
-    const uint32_t b = fastdiv(tok, P.div_t);
-    const int t = (int)(tok - b * (uint32_t)P.T);
+    const uint32_t tok = fastdiv(r, is_q ? P.div_hq : P.div_hkv);  // b * T + t (queries: b * Tq + t)
+    const uint32_t b = fastdiv(tok, is_q ? P.div_tq : P.div_t);
+    const int t = (int)(tok - b * (uint32_t)(is_q ? P.Tq : P.T));
     const __nv_bfloat16* x = (is_q ? q : k) + (size_t)r * D;
     __nv_bfloat16* y = (is_q ? qo : ko) + (size_t)r * D;
     const bool active = valid && g < G::LPR;
@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __rest
         load_bf16x8(x + d0, lo);
         load_bf16x8(x + kHalf + d0, hi);
         if (P.rope) {  // issued together with the row loads: its latency overlaps theirs
-            const int pos = P.seg_start ? t - P.seg_start[tok] : t;
+            // queries over a cache sit at qoff + t; segments only come without a cache
+            const int pos = P.seg_start ? t - P.seg_start[tok] : t + (is_q ? P.qoff : 0);
             const float4* c = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) cs[i] = c[i];
@@ -285,8 +286,8 @@ cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start
 template <int D>
 static cudaError_t launch_prologue_d(const Problem& P, const void* q, const void* k, void* qo, void* ko,
                                      cudaStream_t st) {
-    const long long rows_q = (long long)P.B * P.T * P.Hq;
-    const long long rows = rows_q + (long long)P.B * P.T * P.Hkv;
+    const long long rows_q = (long long)P.B * P.Tq * P.Hq;
+    const long long rows = rows_q + (k ? (long long)P.B * P.T * P.Hkv : 0);  // k == null: queries only
     const long long blocks = (rows + RowGeom<D>::ROWS - 1) / RowGeom<D>::ROWS;
     k_qk_prologue<D><<<(unsigned)blocks, 256, 0, st>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, (uint32_t)rows_q, (uint32_t)rows);

@@ -112,6 +112,16 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
                            const int32_t* segment_ids, void* dq, void* dk, void* dv,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward over a key/value cache (prefill of a chunk of Tq new tokens; "Build and Train a
+ * MiniGPT with JAX", section "Bonus: KV Caching"): the same masking and arguments as
+ * csa_attn_decode below, for any 1 <= Tq <= p->T, on the tensor-core forward.  The cache's
+ * last Tq entries are the new tokens' own keys and values.  Workspace 256-byte aligned and at
+ * least csa_prefill_workspace_size(p, Tq) bytes (0 when the arguments are invalid). */
+size_t csa_prefill_workspace_size(const csa_params* p, int Tq);
+int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_cache,
+                     const void* v_cache, void* o, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
 /* KV-cache decoding ("Build and Train a MiniGPT with JAX", section "Bonus: KV Caching"):
  * Tq new queries attend over a cache of p->T entries.  With offset = p->T - Tq, query i sits
  * at absolute position offset + i and sees cache entry j when j <= offset + i (p->causal = 1;
