@@ -25,6 +25,10 @@
 // written as packed bf16 over the first 64 columns of S_i and fed to the PV MMA from TMEM.
 // MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1): while one softmax group
 // works on its scores the tensor core serves the other one.
+// Epilogue: O (normalised, bf16) goes through one shared staging tile in the TMA box layout
+// and leaves with tiled TMA stores; the two softmax warpgroups take turns on it.
+// Over a key/value cache (chunked prefill) the Tq query rows sit at absolute positions
+// qoff + i, qoff = T - Tq, against the T cached keys; the plain forward has Tq = T, qoff = 0.
 // All mbarrier waits are bounded (see mbar_wait); a wait that runs out records
 // CSA_ERR_DEVICE_TIMEOUT and every role unwinds, frees TMEM and exits.
 #include <cuda.h>
