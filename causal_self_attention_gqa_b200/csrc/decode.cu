@@ -30,10 +30,15 @@ constexpr int kDecThreads = 128;  // 4 warps per CTA
 constexpr int kDecKeysPerCta = 128;  // smallest key range per CTA
 
 // ------------------------------------------------------------------ q prologue
+// RoPE frequencies base^(-2d/D), d < D/2, computed on the host in fp64.
+struct RopeFreq {
+    double theta[64];
+};
+
 // One warp per query row (b, i, h); writes qs[b][kvh][r][d], r = (h % G) * Tq + i.
 template <int D>
 __global__ void __launch_bounds__(128) k_decode_q(const __nv_bfloat16* __restrict__ q, float* __restrict__ qs,
-                                                  Problem P, int Tq) {
+                                                  Problem P, int Tq, const RopeFreq F) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int rows = P.B * Tq * P.Hq;
     if (warp >= rows) return;  // whole warps leave together
@@ -63,8 +68,7 @@ __global__ void __launch_bounds__(128) k_decode_q(const __nv_bfloat16* __restric
             const int d = lane + 32 * t, d2 = d % (D / 2);
             // phase pos * theta in fp64 (it reaches ~1e6 rad), reduced to [-pi, pi] with a
             // two-part 2 pi (Cody-Waite), then the fp32 sine / cosine of the remainder
-            const double theta = exp((-2.0 * d2 / D) * P.rope_log_base);
-            const double phi = (double)pos * theta;
+            const double phi = (double)pos * F.theta[d2];
             const double k = rint(phi * 0.15915494309189535);  // 1 / (2 pi)
             const double red = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, phi));
             float sn, cs;
@@ -284,19 +288,23 @@ __global__ void __launch_bounds__(kDecThreads, RMAX >= 16 ? 2 : 4) k_decode_spli
 }
 
 // ------------------------------------------------------------------ host side
-// Key ranges per (b, kv head): about eight CTAs per SM (latency hiding: each CTA has only
-// four warps), at least 128 keys each.
+// Key ranges for `resident` CTAs per SM: one wave of the grid, at least 128 keys per range.
+// The workspace is sized for resident = 8, the most any launch uses.
+static void split_keys(const Problem& P, int resident, int& splits, int& keys_per_split) {
+    const int ctas = P.B * P.Hkv;
+    int s = ctas > 0 ? resident * num_sms() / ctas : 1;
+    const int max_s = (P.T + kDecKeysPerCta - 1) / kDecKeysPerCta;
+    s = s < 1 ? 1 : (s > max_s ? max_s : s);
+    const int kps = (P.T + s - 1) / s;
+    keys_per_split = (kps + 31) / 32 * 32;
+    splits = (P.T + keys_per_split - 1) / keys_per_split;
+}
+
 DecodePlan decode_plan(const Problem& P, int Tq) {
     DecodePlan d;
     d.Tq = Tq;
     d.R = P.G * Tq;
-    const int ctas = P.B * P.Hkv;
-    int s = ctas > 0 ? (8 * num_sms() + ctas - 1) / ctas : 1;
-    const int max_s = (P.T + kDecKeysPerCta - 1) / kDecKeysPerCta;
-    s = s < 1 ? 1 : (s > max_s ? max_s : s);
-    int kps = (P.T + s - 1) / s;
-    d.keys_per_split = (kps + 31) / 32 * 32;
-    d.splits = (P.T + d.keys_per_split - 1) / d.keys_per_split;
+    split_keys(P, 8, d.splits, d.keys_per_split);
     d.qs_bytes = (size_t)P.B * P.Hkv * d.R * P.D * sizeof(float);
     d.part_bytes = (size_t)P.B * P.Hkv * d.splits * d.R * (P.D + 2) * sizeof(float);
     d.done_bytes = (size_t)P.B * P.Hkv * sizeof(int);
@@ -321,8 +329,22 @@ static DecArgs dec_args(const Problem& P, const DecodePlan& d, const float* qs, 
     return A;
 }
 
+// The grid is one wave: as many key ranges as the SMs hold CTAs of this instance at once
+// (never more than the workspace was sized for).
 template <int D, int RMAX, bool CAP>
-static cudaError_t launch_split(const DecArgs& A, cudaStream_t st) {
+static cudaError_t launch_split(DecArgs A, cudaStream_t st) {
+    static int resident = 0;
+    if (!resident) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_split<D, RMAX, CAP>, kDecThreads, 0) !=
+                cudaSuccess ||
+            n < 1) {
+            cudaGetLastError();
+            n = 4;
+        }
+        resident = n < 8 ? n : 8;
+    }
+    split_keys(A.P, resident, A.splits, A.keys_per_split);
     dim3 grid(A.splits, A.P.Hkv, A.P.B);
     k_decode_split<D, RMAX, CAP><<<grid, kDecThreads, 0, st>>>(A);
     return cudaGetLastError();
@@ -348,8 +370,10 @@ static cudaError_t launch_split_r(const DecArgs& A, cudaStream_t st) {
 cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q, float* qs, cudaStream_t st) {
     const int rows = P.B * d.Tq * P.Hq;
     const int blocks = (rows + 3) / 4;
+    RopeFreq F;
+    for (int i = 0; i < P.D / 2; ++i) F.theta[i] = P.rope ? exp((-2.0 * i / P.D) * P.rope_log_base) : 0.0;
 #define CALL(D_)                                                                                              \
-    (k_decode_q<D_><<<blocks, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qs, P, d.Tq), cudaGetLastError())
+    (k_decode_q<D_><<<blocks, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qs, P, d.Tq, F), cudaGetLastError())
     CSA_DEC_DISPATCH(CALL)
 #undef CALL
 }
