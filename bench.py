@@ -602,6 +602,9 @@ def main():
         "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
         "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None,
         "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd, "pairs_per_head": pairs},
+        # the common convention that counts causal attention as half of dense: 14 D Hq B T^2 / 2
+        "tflops_causal_half_dense": (14.0 * wr.D * wr.Hq * wr.B * world * wr.T * wr.T / 2)
+        / (ms_per_step * 1e-3) / 1e12,
         "kernels": per_kernel,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
     }
