@@ -29,9 +29,21 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_reject_mutant(name, tmp_path):
-    old, new = MUTANTS[name]
+# Mistakes in the KV-cache attention (oracle_attn_fwd_cached), against its own pins.
+CACHED_MUTANTS = {
+    "cached_position_from_zero": ("const int pos = offset + i;", "const int pos = i;"),
+    "cached_mask_off_by_one": ("if (p->causal && j > pos) vis = 0;", "if (p->causal && j >= pos) vis = 0;"),
+    "cached_window_off_by_one": ("if (dd >= p->window || (!p->causal && -dd >= p->window)) vis = 0;",
+                                 "if (dd > p->window || (!p->causal && -dd >= p->window)) vis = 0;"),
+    "cached_gqa_interleaved": ("            const int kvh = h / G;\n            double* qp = (double*)malloc(sizeof(double) * (size_t)D);",
+                               "            const int kvh = h % Hkv;\n            double* qp = (double*)malloc(sizeof(double) * (size_t)D);"),
+    "cached_cap_missing": ("if (p->softcap > 0.0) acc = p->softcap * tanh(acc / p->softcap);", ""),
+    "cached_lse_missing_max": ("lse[((size_t)b * Hq + h) * Tq + i] = m + log(l);",
+                               "lse[((size_t)b * Hq + h) * Tq + i] = log(l);"),
+}
+
+
+def _run_pins(name, old, new, pin_file, tmp_path):
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation anchor for {name} not unique/found"
     mutated = tmp_path / "oracle.c"
@@ -40,7 +52,20 @@ def test_pins_reject_mutant(name, tmp_path):
     subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
                            str(mutated), "-o", str(lib), "-lm"])
     env = dict(os.environ, ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           os.path.join(ROOT, "tests", pin_file)],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+@pytest.mark.parametrize("name", sorted(CACHED_MUTANTS))
+def test_cached_pins_reject_mutant(name, tmp_path):
+    old, new = CACHED_MUTANTS[name]
+    r = _run_pins(name, old, new, "test_oracle_cached.py", tmp_path)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_reject_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    r = _run_pins(name, old, new, "test_oracle.py", tmp_path)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
