@@ -14,12 +14,15 @@
  * section "Multihead Attention"; grouped-query heads, RoPE, QK-norm (parameter-free
  * RMSNorm), logits soft-capping and RoPE from packed segment positions come from the
  * nanogpt-jax-181m model card, section "Architecture", and packed rows with segment_ids
- * from its section "SFT"; the sliding window from the flaxchat README, "Core Features".
+ * from its section "SFT"; the sliding window from the flaxchat README, "Core Features";
+ * attention of new queries over a key/value cache from "Build and Train a MiniGPT with JAX",
+ * section "Bonus: KV Caching".
  * The pages give no formulas for RoPE, the norm, the cap or the window; the readings used
  * here are stated at each field of csa_params.
  *
  * Conventions shared by every entry point
- *  - Tensors are row-major and contiguous: q, o, dout, dq are [B, T, Hq, D] bf16;
+ *  - Tensors are row-major and contiguous (the KV-cache calls state their own query length):
+ *    q, o, dout, dq are [B, T, Hq, D] bf16;
  *    k, v, dk, dv are [B, T, Hkv, D] bf16; lse is [B, Hq, T] fp32; segment_ids is [B, T] int32.
  *    bf16 pointers are passed as void* and hold IEEE bfloat16 bit patterns.
  *  - Every tensor pointer is a DEVICE pointer, allocated and owned by the caller, aligned to
