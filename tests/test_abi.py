@@ -122,3 +122,22 @@ def test_decode_arguments_are_checked_on_the_host(b):
     assert dec(ctypes.byref(p), 1, 0x1008, *ptr[1:5], 0x10000, 1 << 30, None) == b.CSA_ERR_ALIGNMENT
     assert dec(ctypes.byref(p), 1, *ptr[:5], 0x10000, 64, None) == b.CSA_ERR_WORKSPACE
     assert dec(ctypes.byref(p), 1, None, *ptr[1:5], 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
+
+
+def test_prefill_arguments_are_checked_on_the_host(b):
+    """csa_attn_prefill: the chunk length, alignment and workspace size are rejected before
+    anything is enqueued (fake pointers: every call here fails a check)."""
+    p = b.make_params(2, 512, 8, 4, 96, rope_base=10000.0, qk_norm=True)
+    n = b.prefill_workspace_size(p, 128)
+    assert n > 0
+    # RoPE table for the 512 cache positions plus q' of the 128-token chunk
+    assert n >= 512 * 48 * 8 + 2 * 128 * 8 * 96 * 2
+    assert b.prefill_workspace_size(p, 0) == 0
+    assert b.prefill_workspace_size(p, 513) == 0
+    assert b.prefill_workspace_size(b.make_params(2, 512, 8, 4, 96), 128) < n  # no prologue, no table
+    pre = b.lib.csa_attn_prefill
+    ptr = [0x1000 * (i + 1) for i in range(6)]
+    assert pre(ctypes.byref(p), 513, *ptr[:5], 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
+    assert pre(ctypes.byref(p), 128, *ptr[:4], 0x5002, 0x10000, 1 << 30, None) == b.CSA_ERR_ALIGNMENT
+    assert pre(ctypes.byref(p), 128, *ptr[:5], 0x10000, n - 1, None) == b.CSA_ERR_WORKSPACE
+    assert pre(ctypes.byref(p), 128, *ptr[:4], None, 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
