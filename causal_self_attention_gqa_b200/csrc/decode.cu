@@ -1,7 +1,8 @@
 // decode.cu -- attention of a few new queries over a key/value cache (KV-cache decoding).
 //
-// "Build and Train a MiniGPT with JAX", section "Bonus: KV Caching": generation feeds only the
-// new token(s); their queries attend over the cached keys and values of the whole history.
+// GPT-pretraining post (dekermanjian.github.io, llm_gpt_pretrain), section "Bonus: KV Caching":
+// generation feeds only the new token(s); their queries attend over the cached keys and
+// values of the whole history.
 // With Tk cached entries and Tq new queries, offset = Tk - Tq and query i sits at absolute
 // position offset + i: it sees key j only when j <= offset + i (and, with a window W, when
 // offset + i - j < W).  The cache holds keys as stored after their own QK-norm and RoPE; the

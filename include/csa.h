@@ -15,8 +15,8 @@
  * RMSNorm), logits soft-capping and RoPE from packed segment positions come from the
  * nanogpt-jax-181m model card, section "Architecture", and packed rows with segment_ids
  * from its section "SFT"; the sliding window from the flaxchat README, "Core Features";
- * attention of new queries over a key/value cache from "Build and Train a MiniGPT with JAX",
- * section "Bonus: KV Caching".
+ * attention of new queries over a key/value cache from the GPT-pretraining page, section
+ * "Bonus: KV Caching".
  * The pages give no formulas for RoPE, the norm, the cap or the window; the readings used
  * here are stated at each field of csa_params.
  *
@@ -115,8 +115,8 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
                            const int32_t* segment_ids, void* dq, void* dk, void* dv,
                            void* workspace, size_t workspace_bytes, void* stream);
 
-/* Forward over a key/value cache (prefill of a chunk of Tq new tokens; "Build and Train a
- * MiniGPT with JAX", section "Bonus: KV Caching"): the same masking and arguments as
+/* Forward over a key/value cache (prefill of a chunk of Tq new tokens; the GPT-pretraining
+ * page (dekermanjian.github.io, llm_gpt_pretrain), section "Bonus: KV Caching"): the same masking and arguments as
  * csa_attn_decode below, for any 1 <= Tq <= p->T, on the tensor-core forward.  The cache's
  * last Tq entries are the new tokens' own keys and values.  Workspace 256-byte aligned and at
  * least csa_prefill_workspace_size(p, Tq) bytes (0 when the arguments are invalid). */
@@ -125,7 +125,8 @@ int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_c
                      const void* v_cache, void* o, float* lse, void* workspace,
                      size_t workspace_bytes, void* stream);
 
-/* KV-cache decoding ("Build and Train a MiniGPT with JAX", section "Bonus: KV Caching"):
+/* KV-cache decoding (the GPT-pretraining page, dekermanjian.github.io, llm_gpt_pretrain,
+ * section "Bonus: KV Caching"):
  * Tq new queries attend over a cache of p->T entries.  With offset = p->T - Tq, query i sits
  * at absolute position offset + i and sees cache entry j when j <= offset + i (p->causal = 1;
  * 0: every entry) and, with a window W > 0, when |offset + i - j| < W.

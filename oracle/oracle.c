@@ -342,7 +342,8 @@ int oracle_attn_bwd(const oracle_params* p, const double* q, const double* k, co
 }
 
 /* Attention of Tq new queries over a key/value cache of p->T entries (KV-cache decoding):
- * "Build and Train a MiniGPT with JAX", section "Bonus: KV Caching".  The new queries are
+ * the GPT-pretraining post (dekermanjian.github.io, llm_gpt_pretrain), section "Bonus: KV
+ * Caching".  The new queries are
  * the last Tq positions of the sequence: offset = T - Tq, and query i sits at absolute
  * position offset + i, so it may see key j only when j <= offset + i (causal); with a
  * window also offset + i - j < W.  The cache holds keys as they were stored after their own

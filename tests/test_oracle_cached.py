@@ -1,7 +1,7 @@
-"""Pins of the oracle's KV-cache attention (oracle_attn_fwd_cached), following "Build and
-Train a MiniGPT with JAX", section "Bonus: KV Caching": Tq new queries at absolute positions
-offset + i, offset = Tk - Tq, over the cached keys and values; a key j is visible to query i
-when j <= offset + i.
+"""Pins of the oracle's KV-cache attention (oracle_attn_fwd_cached), following the
+GPT-pretraining post (dekermanjian.github.io, llm_gpt_pretrain), section "Bonus: KV Caching":
+Tq new queries at absolute positions offset + i, offset = Tk - Tq, over the cached keys and
+values; a key j is visible to query i when j <= offset + i.
 
 The cached computation takes its keys already normalised and rotated (as the prologue stores
 them) and applies the norm and RoPE to the queries at their absolute positions.  It must give
