@@ -4,9 +4,10 @@ Tolerances (stated for the bf16 path): O relative L2 <= 1e-2 and max-abs <= 2e-2
 dQ, dK, dV relative L2 <= 2e-2 each; LSE max-abs <= 1e-2 (internal).
 Small shapes cover every option, ragged tails (T not a multiple of the 128-row tile),
 T = 1, odd group sizes and windows that bind.  The named workloads run at full size
-in the launch configuration the benchmark times, checked against the oracle on sampled
-batch rows (batch rows are independent, so a row's outputs and gradients are exact
-oracle targets).
+in the call sequence and launch configuration the benchmark times (forward, then the
+backward that reuses the forward's workspace): O and LSE on every batch row, gradients per
+head on the first, middle and last rows (batch rows are independent, so a row's outputs and
+gradients are exact oracle targets).
 """
 import numpy as np
 import pytest
@@ -95,6 +96,9 @@ SMALL = [
     (2, 200, 4, 2, 64, dict(rope_base=10000.0, qk_norm=True), None),
     (1, 300, 2, 1, 128, dict(rope_base=10000.0, qk_norm=True, softcap=50.0), None),
     (1, 300, 2, 1, 64, dict(softcap=5.0), None),            # cap that binds (no norm)
+    # QK-norm with a cap too tight for the series tanh (D scale / cap > 1/4): hardware tanh
+    (1, 300, 4, 2, 128, dict(rope_base=10000.0, qk_norm=True, softcap=20.0), None),
+    (2, 200, 2, 1, 64, dict(qk_norm=True, softcap=50.0), None),  # series tanh at D = 64
     (1, 520, 2, 1, 96, dict(window=100), None),             # window that binds, ragged
     (2, 384, 4, 2, 128, dict(rope_base=10000.0, qk_norm=True, window=200), (20, 150)),
     (1, 300, 2, 2, 32, dict(), (1, 40)),                    # segments, single-token documents
@@ -117,12 +121,12 @@ def test_small_shapes_match_oracle(csa, ora, case):
     check(gpu, ref_o, ref_lse, ref_g)
 
 
-@pytest.mark.parametrize("case", [SMALL[i] for i in (2, 8, 10, 13, 17)],
+@pytest.mark.parametrize("case", [SMALL[i] for i in (2, 8, 10, 12, 15, 19)],
                          ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}x{c[3]}D{c[4]}"
                          + "".join(f"-{k}{v}" for k, v in c[5].items()) + ("-seg" if c[6] else ""))
 def test_backward_after_forward_reuses_the_workspace(csa, ora, case):
-    """csa_attn_bwd_after_fwd (q', k', segment bounds and RoPE table from the forward's
-    workspace, no prologue) against the oracle: with and without norm / RoPE / segments."""
+    """csa_attn_bwd_after_fwd (q', k' and segment bounds from the forward's workspace, no
+    prologue) against the oracle: with and without norm / RoPE / segments."""
     B, T, Hq, Hkv, D, opts, seg = case
     w, inp = _small(B, T, Hq, Hkv, D, seed=11 + T + D, seg=seg, **opts)
     kw = dict(w.options())
@@ -132,23 +136,58 @@ def test_backward_after_forward_reuses_the_workspace(csa, ora, case):
     check(gpu, ref_o, ref_lse, ref_g)
 
 
+def grad_rows(w):
+    """Batch rows whose gradients the full-size tests compare: first, middle and last."""
+    return sorted({0, w.B // 2, w.B - 1})
+
+
+def check_per_head(name, got, ref, tol):
+    """Relative L2 per (batch row, head) of [rows, T, H, D] gradients: a single wrong head
+    cannot hide inside a norm taken over the whole tensor."""
+    assert np.all(np.isfinite(got)), name
+    for r in range(got.shape[0]):
+        for h in range(got.shape[2]):
+            e = rel_l2(got[r, :, h], ref[r, :, h])
+            assert e <= tol, (name, r, h, e)
+
+
 @pytest.mark.parametrize("widx", range(len(WORKLOADS)), ids=[w.name for w in WORKLOADS])
-def test_workload_full_size_sampled_rows(csa, ora, widx):
-    """Full-size run (the benchmark's launch configuration); oracle on sampled batch rows."""
+def test_benchmarked_step_full_size(csa, ora, widx):
+    """The exact sequence the benchmark times, at full size: csa_attn_fwd, then
+    csa_attn_bwd_after_fwd on the same workspace (q', k', segment bounds and whatever else
+    the forward left there).  O and LSE are compared with the oracle on EVERY batch row;
+    dQ, dK, dV on the first, middle and last rows, per head."""
+    w = WORKLOADS[widx]
+    inp = make_inputs(w)
+    kw = dict(w.options())
+    gpu = run_gpu(csa, inp, kw, after_fwd=True)
+    ref_o, ref_lse = ora.attn_fwd(inp["q"], inp["k"], inp["v"], segment_ids=inp["segment_ids"], **kw)
+    for b in range(w.B):
+        check(gpu, ref_o[b:b + 1], ref_lse[b:b + 1], rows=slice(b, b + 1))
+    rows = grad_rows(w)
+    seg = inp["segment_ids"][rows] if inp["segment_ids"] is not None else None
+    ref_g = ora.attn_bwd(inp["q"][rows], inp["k"][rows], inp["v"][rows], inp["do"][rows], segment_ids=seg, **kw)
+    for name, ref in zip(("dq", "dk", "dv"), ref_g):
+        check_per_head(name, gpu[name][rows], ref, G_REL)
+
+
+@pytest.mark.parametrize("widx", range(len(WORKLOADS)), ids=[w.name for w in WORKLOADS])
+def test_stateless_backward_full_size(csa, ora, widx):
+    """csa_attn_bwd (the stateless backward, which reruns the prologue itself) at full size,
+    against the oracle on the last batch row, per head."""
     w = WORKLOADS[widx]
     inp = make_inputs(w)
     kw = dict(w.options())
     gpu = run_gpu(csa, inp, kw)
-    rows = [0] if w.B <= 2 else [0, w.B - 1]
-    if w.T <= 128:
-        rows = list(range(w.B))
-    for b in rows:
-        sl = slice(b, b + 1)
-        seg = inp["segment_ids"][sl] if inp["segment_ids"] is not None else None
-        args = (inp["q"][sl], inp["k"][sl], inp["v"][sl])
-        ref_o, ref_lse = ora.attn_fwd(*args, segment_ids=seg, **kw)
-        ref_g = ora.attn_bwd(*args, inp["do"][sl], segment_ids=seg, **kw)
-        check(gpu, ref_o, ref_lse, ref_g, rows=sl)
+    b = w.B - 1
+    sl = slice(b, b + 1)
+    seg = inp["segment_ids"][sl] if inp["segment_ids"] is not None else None
+    args = (inp["q"][sl], inp["k"][sl], inp["v"][sl])
+    ref_o, ref_lse = ora.attn_fwd(*args, segment_ids=seg, **kw)
+    check(gpu, ref_o, ref_lse, rows=sl)
+    ref_g = ora.attn_bwd(*args, inp["do"][sl], segment_ids=seg, **kw)
+    for name, ref in zip(("dq", "dk", "dv"), ref_g):
+        check_per_head(name, gpu[name][sl], ref, G_REL)
 
 
 def test_causal_outputs_ignore_future_tokens(csa):
