@@ -18,6 +18,11 @@ with an L2 flush (256 MiB write) between steps outside the events; a barrier and
 device synchronize on both sides; the max over ranks.  With N > 1 every rank runs its own
 batch (independent problems, weak scaling); the only collective is the timing reduction.
 `--impl reference` times the fp64 CPU oracle (the reference arm) on a bounded sample.
+
+At N = 1 the line also carries `per_workload`: the same step, steps and warm-up for every
+named workload (ms/step, TFLOP/s, tokens/s, % of the measured burst peak, forward and
+backward kernel TFLOP/s, kernel shares), plus the KV-cache decode leg (GB/s against HBM)
+and the chunked-prefill leg (TFLOP/s).
 """
 from __future__ import annotations
 
@@ -200,55 +205,61 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle arm
-def oracle_sample(w, inp, step: int, threads: int):
-    """One bounded sample of the workload on the CPU oracle: one batch row and one
-    key/value head group (its G query heads), forward + backward."""
+def oracle_units(w, start: int, n: int):
+    """The (batch row, key/value-head group) units start .. start+n-1 of the workload, in
+    row-major order (wrapping): the oracle's own work units (its backward runs OpenMP over
+    them, its forward over their query heads)."""
+    total = w.B * w.Hkv
+    return [((start + i) % total // w.Hkv, (start + i) % total % w.Hkv) for i in range(n)]
+
+
+def oracle_sample(w, inp, units, threads: int):
+    """fwd + bwd of the CPU oracle, as it stands, on the given (b, group) units run as one
+    batch on `threads` OpenMP threads.  Returns (TFLOP/s, seconds, FLOPs)."""
     import oracle
     oracle.build()
     oracle.set_threads(threads)
     G = w.Hq // w.Hkv
-    b = step % w.B
-    g = (step // w.B) % w.Hkv
-    sl = slice(b, b + 1)
-    q = inp["q"][sl, :, g * G:(g + 1) * G]
-    k = inp["k"][sl, :, g:g + 1]
-    v = inp["v"][sl, :, g:g + 1]
-    do = inp["do"][sl, :, g * G:(g + 1) * G]
-    seg = inp["segment_ids"][sl] if inp["segment_ids"] is not None else None
+    q = torch.stack([inp["q"][b, :, g * G:(g + 1) * G] for b, g in units])
+    k = torch.stack([inp["k"][b, :, g:g + 1] for b, g in units])
+    v = torch.stack([inp["v"][b, :, g:g + 1] for b, g in units])
+    do = torch.stack([inp["do"][b, :, g * G:(g + 1) * G] for b, g in units])
+    seg = torch.stack([inp["segment_ids"][b] for b, _ in units]) if inp["segment_ids"] is not None else None
     kw = w.options()
     t0 = time.perf_counter()
     oracle.attn_fwd(q, k, v, segment_ids=seg, **kw)
     oracle.attn_bwd(q, k, v, do, segment_ids=seg, **kw)
     dt = time.perf_counter() - t0
-    sub = w.with_(B=1, Hq=G, Hkv=1)
+    sub = w.with_(B=len(units), Hq=G, Hkv=1)
     f, bw, _ = flops(sub, seg.numpy() if seg is not None else None)
     return (f + bw) / dt / 1e12, dt, f + bw
 
 
+def host_cores() -> int:
+    return len(os.sched_getaffinity(0))
+
+
 def run_reference(args, w):
+    """The reference arm: the fp64 oracle on the host's cores.  Step i is the oracle's
+    forward + backward of one (batch row, key/value-head group) unit of the workload; the
+    W warm-up units, then the K timed units, each run as one batch on every core, so the
+    whole run stays within minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     inp = make_inputs(w)
-    cores = len(os.sched_getaffinity(0))
-    threads = min(cores, w.Hq // w.Hkv)
-    for s in range(args.warmup):
-        oracle_sample(w, inp, s, threads)
-    times, fl = [], []
-    for s in range(args.steps):
-        _, dt, f = oracle_sample(w, inp, args.warmup + s, threads)
-        times.append(dt)
-        fl.append(f)
-    value = sum(fl) / sum(times) / 1e12
-    sample = (f"one batch row x one KV-head group ({w.Hq // w.Hkv} query heads) of {w.name} per step, "
-              f"fwd+bwd, fp64")
+    cores = host_cores()
+    oracle_sample(w, inp, oracle_units(w, 0, max(args.warmup, 1)), cores)
+    value, dt, _ = oracle_sample(w, inp, oracle_units(w, args.warmup, args.steps), cores)
+    sample = (f"{args.steps} units of one batch row x one KV-head group ({w.Hq // w.Hkv} query heads) of "
+              f"{w.name}, fwd+bwd in fp64, run as one batch on {cores} threads")
     line = {"impl": "reference", "metric": metric_name(), "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(w, args.gpus),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "threads": cores,
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -285,14 +296,14 @@ def profile_step(w):
     return 0 if rc == 0 else 1
 
 
-def run_decode(args):
+def measure_decode(steps: int, warmup: int, batch: int = 0) -> dict:
     """KV-cache decoding (csa_attn_decode), 1 GPU: cache bytes read per second against the
     measured HBM copy bandwidth.  The K/V cache (201 MB at the default shape) is larger than
     L2, so every step streams it from HBM; no flush is needed between steps."""
     from causal_self_attention_gqa_b200 import _binding as csa
     w = DECODE_WORKLOADS[0]
-    if args.batch > 0:
-        w = w.with_(B=args.batch)
+    if batch > 0:
+        w = w.with_(B=batch)
     dev = torch.device("cuda:0")
     inp = make_decode_inputs(w)
     q, kc, vc = (inp[n].to(dev) for n in ("q", "k_cache", "v_cache"))
@@ -302,7 +313,7 @@ def run_decode(args):
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         csa.attn_decode(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
     torch.cuda.synchronize()
     rc = csa.device_status(ws)
@@ -311,43 +322,42 @@ def run_decode(args):
     csa.timing_enable(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         csa.attn_decode(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
     e1.record(stream)
     torch.cuda.synchronize()
     csa.timing_enable(False)
     kt = csa.timing_collect()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
     cache_bytes = 2 * w.B * w.Tk * w.Hkv * w.D * 2
     io_bytes = cache_bytes + 2 * q.numel() * 2 + lse.numel() * 4
     peaks, src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    split_ms = kt["k_decode_split"][0] / max(kt["k_decode_split"][1], 1)
+    split_ms = kt["k_decode"][0] / max(kt["k_decode"][1], 1)
     gbs = io_bytes / (ms * 1e-3) / 1e9
     split_gbs = cache_bytes / (split_ms * 1e-3) / 1e9
     line = {
         "metric": "KV-cache decode step: bytes read per second (cache + queries + outputs)", "value": gbs,
-        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": max(warmup, 3), "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see workloads.py)",
         "config": {"workload": w.name, "B": w.B, "Tk": w.Tk, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "options": kw, "l2": "cache larger than L2, streamed every step"},
         "tokens_per_s": w.B * w.Tq / (ms * 1e-3),
         "kernels": {n: {"ms_avg": t / c if c else 0.0, "launches": c} for n, (t, c) in kt.items() if c},
         "roofline": {"bound": "hbm", "achieved": split_gbs, "peak": hbm, "unit": "GB/s", "frac": split_gbs / hbm,
-                     "traffic": None, "kernel": "k_decode_split", "peak_source": f"{src}, hbm_gbs"},
+                     "traffic": None, "kernel": "k_decode", "peak_source": f"{src}, hbm_gbs"},
         "gpu_launches": sum(c for _, c in kt.values()),
     }
-    print(json.dumps(line))
-    return 0
+    return line
 
 
-def run_prefill(args):
+def measure_prefill(steps: int, warmup: int, batch: int = 0) -> dict:
     """Forward over a KV cache (csa_attn_prefill): a 2048-token chunk at the end of an
     8192-entry cache, 181M shape, batch 4; algorithmic TFLOP/s (4 D per visible pair and query
     head) against the measured bf16 peak.  The caches (101 MB) and queries exceed L2 together."""
     from causal_self_attention_gqa_b200 import _binding as csa
     from causal_self_attention_gqa_b200.workloads import DecodeWorkload
-    w = DecodeWorkload("prefill_gpt181m_gqa8x4_D96_rope_qknorm_chunk2048_cache8192", B=args.batch or 4, Tk=8192,
+    w = DecodeWorkload("prefill_gpt181m_gqa8x4_D96_rope_qknorm_chunk2048_cache8192", B=batch or 4, Tk=8192,
                        Tq=2048, Hq=8, Hkv=4, D=96, rope_base=10000.0, qk_norm=True, seed=2001)
     dev = torch.device("cuda:0")
     inp = make_decode_inputs(w)
@@ -359,7 +369,7 @@ def run_prefill(args):
     lse = torch.empty((w.B, w.Hq, w.Tq), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         csa.attn_prefill(q, kc, vc, out=o, lse=lse, workspace=ws, **kw)
     torch.cuda.synchronize()
     rc = csa.device_status(ws)
@@ -367,7 +377,7 @@ def run_prefill(args):
         raise RuntimeError(f"device status after warm-up: {csa.status_string(rc)}")
     csa.timing_enable(True)
     times = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -377,7 +387,7 @@ def run_prefill(args):
     torch.cuda.synchronize()
     csa.timing_enable(False)
     kt = {n: tc for n, tc in csa.timing_collect().items() if tc[1] > 0}
-    ms = sum(a.elapsed_time(b) for a, b in times) / args.steps
+    ms = sum(a.elapsed_time(b) for a, b in times) / steps
     off = w.Tk - w.Tq
     pairs = sum(off + i + 1 for i in range(w.Tq))  # causal, per (b, query head)
     flops = 4.0 * w.D * w.Hq * w.B * pairs
@@ -386,7 +396,7 @@ def run_prefill(args):
     fwd_ms = kt["k_attn_fwd"][0] / kt["k_attn_fwd"][1]
     line = {
         "metric": "forward over a KV cache (chunked prefill): algorithmic TFLOP/s", "value": flops / (ms * 1e-3) / 1e12,
-        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": max(warmup, 3), "ms_per_step": ms,
         "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; see workloads.py)",
         "config": {"workload": w.name, "B": w.B, "Tk": w.Tk, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "options": kw, "l2": "flushed between timed steps (256 MiB write, outside the events)"},
@@ -397,8 +407,63 @@ def run_prefill(args):
                      "peak_source": f"{src}, bf16_tflops"},
         "gpu_launches": sum(c for _, c in kt.values()),
     }
-    print(json.dumps(line))
-    return 0
+    return line
+
+
+def measure_training(w, dev, steps: int, warmup: int, flush) -> dict:
+    """The training step (csa_attn_fwd, then csa_attn_bwd_after_fwd on the same workspace) of
+    workload w on one GPU, timed like the headline: per-step CUDA events, L2 flush between
+    steps outside the events, per-kernel library events in the same region."""
+    from causal_self_attention_gqa_b200 import _binding as csa
+    inp = make_inputs(w)
+    seg_np = inp["segment_ids"].numpy() if inp["segment_ids"] is not None else None
+    f_fwd, f_bwd, pairs = flops(w, seg_np)
+    kw = w.options()
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    seg = inp["segment_ids"].to(dev) if inp["segment_ids"] is not None else None
+    ws = csa.workspace_for(q, k, True, **kw)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.attn_fwd(q, k, v, segment_ids=seg, out=o, lse=lse, workspace=ws, **kw)
+        csa.attn_bwd(q, k, v, o, do, lse, segment_ids=seg, dq=dq, dk=dk, dv=dv, workspace=ws, after_fwd=True,
+                     **kw)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"{w.name}: device status after warm-up: {csa.status_string(rc)}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    csa.timing_enable(True)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    csa.timing_enable(False)
+    kt = {n: tc for n, tc in csa.timing_collect().items() if tc[1] > 0}
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"{w.name}: device status after the timed steps: {csa.status_string(rc)}")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tot_k = sum(t for t, _ in kt.values()) or 1.0
+    fwd_ms = kt["k_attn_fwd"][0] / kt["k_attn_fwd"][1]
+    bwd_ms = kt["k_attn_bwd"][0] / kt["k_attn_bwd"][1]
+    tflops = (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+    return {"ms_per_step": ms, "tflops": tflops, "tokens_per_s": w.B * w.T / (ms * 1e-3),
+            "pct_of_measured_burst": 100.0 * tflops / peak,
+            "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+            "flops_per_step": f_fwd + f_bwd, "pairs_per_head": pairs, "steps": steps, "warmup": max(warmup, 3),
+            "launches_per_step": sum(c for _, c in kt.values()) / steps,
+            "kernels": {n: {"ms_avg": t / c, "share": t / tot_k} for n, (t, c) in kt.items()}}
 
 
 def main():
@@ -409,6 +474,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-workload map (every named workload, decode and prefill legs)")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end leg (default: min(K, 20))")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling cases)")
     ap.add_argument("--prefill", action="store_true",
@@ -424,9 +491,11 @@ def main():
     if args.profile_step:
         return profile_step(w)
     if args.decode:
-        return run_decode(args)
+        print(json.dumps(measure_decode(args.steps, args.warmup, args.batch)))
+        return 0
     if args.prefill:
-        return run_prefill(args)
+        print(json.dumps(measure_prefill(args.steps, args.warmup, args.batch)))
+        return 0
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -578,14 +647,40 @@ def main():
                "ms_per_step": e_ms / n_e2e,
                "copies": "pinned host buffers, one stream per direction, two device slots (overlapped with compute)"}
 
+    # every named workload (same steps, warm-up and timing), then the KV-cache legs; one GPU
+    per_workload = None
+    if world == 1 and not args.no_per_workload:
+        per_workload = {}
+        for wk in WORKLOADS:
+            if wk.name == wr.name:
+                per_workload[wk.name] = {
+                    "ms_per_step": ms_per_step, "tflops": value, "tokens_per_s": tokens_per_s,
+                    "pct_of_measured_burst": 100.0 * value / float(load_peaks()[0].get("bf16_tflops", 1.0)),
+                    "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+                    "flops_per_step": f_fwd + f_bwd, "pairs_per_head": pairs, "steps": args.steps,
+                    "warmup": max(args.warmup, 3), "launches_per_step": launches / args.steps,
+                    "kernels": {n: {"ms_avg": d["ms_avg"], "share": d["share"]} for n, d in per_kernel.items()},
+                    "headline": True}
+            else:
+                per_workload[wk.name] = measure_training(wk, dev, args.steps, args.warmup, flush)
+        dl = measure_decode(args.steps, args.warmup)
+        per_workload[dl["config"]["workload"]] = {
+            "ms_per_step": dl["ms_per_step"], "gbs": dl["value"], "tokens_per_s": dl["tokens_per_s"],
+            "roofline": dl["roofline"], "kernels": dl["kernels"], "steps": dl["steps"], "warmup": dl["warmup"]}
+        pl = measure_prefill(args.steps, args.warmup)
+        per_workload[pl["config"]["workload"]] = {
+            "ms_per_step": pl["ms_per_step"], "tflops": pl["value"], "tokens_per_s": pl["tokens_per_s"],
+            "roofline": pl["roofline"], "kernels": pl["kernels"], "steps": pl["steps"], "warmup": pl["warmup"]}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = len(os.sched_getaffinity(0))
-        threads = min(cores, wr.Hq // wr.Hkv)
-        val, dt, _ = oracle_sample(wr, inp, 0, threads)
-        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"one batch row x one KV-head group ({wr.Hq // wr.Hkv} query heads) of {wr.name}, "
-                         f"fwd+bwd in fp64, {dt:.1f} s"}
+        # one unit per core, so every core works: about one unit's time (10-30 s at T = 2048)
+        cores = host_cores()
+        units = oracle_units(wr, 0, cores)
+        val, dt, _ = oracle_sample(wr, inp, units, cores)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cores, "threads": cores, "kind": "oracle",
+               "sample": f"{len(units)} units of one batch row x one KV-head group ({wr.Hq // wr.Hkv} query heads) "
+                         f"of {wr.name}, fwd+bwd in fp64 on {cores} threads, {dt:.1f} s"}
 
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -607,6 +702,7 @@ def main():
         / (ms_per_step * 1e-3) / 1e12,
         "kernels": per_kernel,
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        "per_workload": per_workload,
     }
     print(json.dumps(line), flush=True)
     return 0
