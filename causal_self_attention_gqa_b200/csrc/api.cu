@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+#include <utility>
 #include <vector>
 
 #include "csa_internal.h"
@@ -13,8 +15,7 @@
 namespace csa {
 int run_selftest_wait(int* status, void* out, cudaStream_t st);
 size_t selftest_out_bytes();
-cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end, float2* rope_cs,
-                        double rope_base, cudaStream_t st);
+cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end, cudaStream_t st);
 cudaError_t launch_prologue(const Problem& P, const void* q, const void* k, void* qo, void* ko, cudaStream_t st);
 cudaError_t launch_bwd_pre(const Problem& P, const void* o, const void* dout, float* delta, float* dq_acc,
                            cudaStream_t st);
@@ -26,9 +27,8 @@ cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMa
                        const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
                        const float* lse, const float* delta, float* dq_acc, cudaStream_t st);
 DecodePlan decode_plan(const Problem& P, int Tq);
-cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q, float* qs, cudaStream_t st);
-cudaError_t launch_decode_split(const Problem& P, const DecodePlan& d, const float* qs, const void* kc,
-                                const void* vc, float* part, int* done, void* o, float* lse, cudaStream_t st);
+cudaError_t launch_decode(const Problem& P, const DecodePlan& d, const void* q, const CUtensorMap& tk,
+                          const CUtensorMap& tv, float* part, int* done, void* o, float* lse, cudaStream_t st);
 
 int num_sms() {
     static int cache[64] = {0};
@@ -48,6 +48,20 @@ int num_sms() {
     return cache[dev];
 }
 
+cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::vector<std::pair<const void*, int>> done;  // (kernel, device) pairs already set
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto& d : done)
+        if (d.first == kernel && d.second == dev) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.emplace_back(kernel, dev);
+    return e;
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -55,8 +69,7 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-    size_t status = 0, seg_start = 0, seg_end = 0, rope = 0, qp = 0, kp = 0, delta = 0, dq_acc = 0, dk_acc = 0,
-           total = 0;
+    size_t status = 0, seg_start = 0, seg_end = 0, qp = 0, kp = 0, delta = 0, dq_acc = 0, dk_acc = 0, total = 0;
 };
 
 bool needs_prologue(const csa_params& p) { return p.qk_norm != 0 || p.rope_base > 0.f; }
@@ -72,10 +85,6 @@ Layout layout(const csa_params& p, bool backward, bool has_seg) {
         off += up(BT * 4);
         L.seg_end = off;
         off += up(BT * 4);
-    }
-    if (p.rope_base > 0.f) {
-        L.rope = off;
-        off += up((size_t)p.T * (p.D / 2) * 8);
     }
     if (needs_prologue(p)) {
         L.qp = off;
@@ -241,13 +250,18 @@ Problem make_problem(const csa_params& p, int* status) {
     P.scale_log2 = (float)((double)P.scale * 1.4426950408889634);
     P.cap_in = P.softcap > 0.f ? (float)((double)P.scale / (double)P.softcap) : 0.f;
     P.cap_log2 = (float)((double)P.softcap * 1.4426950408889634);
+    // With QK-norm on the prologue's own output, |q'| and |k'| are at most sqrt(D) (RMS at
+    // most 1; bf16 rounding adds below 2^-9 each), so |scale q'.k' / softcap| is at most
+    // D scale / softcap times 1.004; the series tanh serves while that stays under 1/4
+    // (2% margin).  Callers whose keys do not come from the prologue clear the flag.
+    P.cap_series = (P.softcap > 0.f && p.qk_norm &&
+                    (double)p.D * (double)P.scale / (double)P.softcap * 1.02 <= 0.25) ? 1 : 0;
     P.rope = p.rope_base > 0.f ? 1 : 0;
     P.rope_log_base = p.rope_base > 0.f ? log((double)p.rope_base) : 0.0;
     P.qk_norm = p.qk_norm;
     P.eps = p.qk_norm_eps;
     P.seg_start = nullptr;
     P.seg_end = nullptr;
-    P.rope_cs = nullptr;
     P.div_hq = make_fastdiv((uint32_t)p.Hq);
     P.div_hkv = make_fastdiv((uint32_t)p.Hkv);
     P.div_t = make_fastdiv((uint32_t)(p.T > 0 ? p.T : 1));
@@ -259,7 +273,7 @@ Problem make_problem(const csa_params& p, int* status) {
     return P;
 }
 
-// Shared front half of both calls: checks, status reset, segments, RoPE table, prologue.
+// Shared front half of both calls: checks, status reset, segment bounds, prologue.
 struct Prepared {
     Problem P;
     Layout L;
@@ -267,8 +281,8 @@ struct Prepared {
     const void* qk_k;
 };
 
-// reuse: the forward already left the segment bounds, the RoPE table and q', k' in the same
-// workspace (same layout: the backward only appends); nothing is launched but the reset.
+// reuse: the forward already left the segment bounds and q', k' in the same workspace (same
+// layout: the backward only appends); nothing is launched but the reset.
 int prepare(const csa_params* p, bool backward, const void* q, const void* k, const int32_t* seg, void* ws,
             size_t ws_bytes, cudaStream_t st, Prepared& out, bool reuse = false) {
     const bool has_seg = seg != nullptr;
@@ -283,17 +297,15 @@ int prepare(const csa_params* p, bool backward, const void* q, const void* k, co
     }
     int32_t* ss = has_seg ? reinterpret_cast<int32_t*>(w + out.L.seg_start) : nullptr;
     int32_t* se = has_seg ? reinterpret_cast<int32_t*>(w + out.L.seg_end) : nullptr;
-    float2* rope = p->rope_base > 0.f ? reinterpret_cast<float2*>(w + out.L.rope) : nullptr;
     out.P.seg_start = ss;
     out.P.seg_end = se;
-    out.P.rope_cs = rope;
     if (reuse) {
         out.qk_q = needs_prologue(*p) ? static_cast<const void*>(w + out.L.qp) : q;
         out.qk_k = needs_prologue(*p) ? static_cast<const void*>(w + out.L.kp) : k;
         return CSA_OK;
     }
-    if (has_seg || rope) {
-        const int rc = timed(kPrep, st, [&] { return launch_prep(out.P, seg, ss, se, rope, p->rope_base, st); });
+    if (has_seg) {
+        const int rc = timed(kPrep, st, [&] { return launch_prep(out.P, seg, ss, se, st); });
         if (rc) return rc;
     }
     out.qk_q = q;
@@ -403,7 +415,7 @@ int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, co
 // ------------------------------------------------------------------ forward over a KV cache
 // Tq queries at absolute positions T - Tq + i over a cache of p->T entries (chunked prefill);
 // the tensor-core forward with its own query length and offset.  Workspace: status slot,
-// RoPE table (positions 0..T-1), q' (queries only: the cache holds processed keys).
+// q' (queries only: the cache holds processed keys).
 static int check_prefill(const csa_params* p, int Tq) {
     int rc = check_params(p);
     if (rc) return rc;
@@ -411,10 +423,8 @@ static int check_prefill(const csa_params* p, int Tq) {
     return CSA_OK;
 }
 
-static size_t prefill_ws_bytes(const csa_params* p, int Tq, size_t* rope_off, size_t* qp_off) {
+static size_t prefill_ws_bytes(const csa_params* p, int Tq, size_t* qp_off) {
     size_t off = kAlign;
-    *rope_off = off;
-    if (p->rope_base > 0.f) off += up((size_t)p->T * (p->D / 2) * 8);
     *qp_off = off;
     if (needs_prologue(*p)) off += up((size_t)p->B * Tq * p->Hq * p->D * 2);
     return off;
@@ -422,8 +432,8 @@ static size_t prefill_ws_bytes(const csa_params* p, int Tq, size_t* rope_off, si
 
 size_t csa_prefill_workspace_size(const csa_params* p, int Tq) {
     if (check_prefill(p, Tq) != CSA_OK) return 0;
-    size_t a, b;
-    return prefill_ws_bytes(p, Tq, &a, &b);
+    size_t a;
+    return prefill_ws_bytes(p, Tq, &a);
 }
 
 int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_cache, const void* v_cache, void* o,
@@ -435,8 +445,8 @@ int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_c
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
         !aligned(workspace, 256))
         return CSA_ERR_ALIGNMENT;
-    size_t rope_off, qp_off;
-    if (workspace_bytes < prefill_ws_bytes(p, Tq, &rope_off, &qp_off)) return CSA_ERR_WORKSPACE;
+    size_t qp_off;
+    if (workspace_bytes < prefill_ws_bytes(p, Tq, &qp_off)) return CSA_ERR_WORKSPACE;
     if ((rc = check_device())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* w = static_cast<uint8_t*>(workspace);
@@ -448,10 +458,7 @@ int csa_attn_prefill(const csa_params* p, int Tq, const void* q, const void* k_c
     P.Tq = Tq;
     P.qoff = p->T - Tq;
     P.div_tq = make_fastdiv((uint32_t)Tq);
-    float2* rope = p->rope_base > 0.f ? reinterpret_cast<float2*>(w + rope_off) : nullptr;
-    P.rope_cs = rope;
-    if (rope && (rc = timed(kPrep, st, [&] { return launch_prep(P, nullptr, nullptr, nullptr, rope, p->rope_base, st); })))
-        return rc;
+    P.cap_series = 0;  // the cached keys come from the caller: no bound on the scores
     const void* qq = q;
     if (needs_prologue(*p)) {
         void* qp = w + qp_off;
@@ -476,10 +483,12 @@ static int check_decode(const csa_params* p, int Tq) {
     return CSA_OK;
 }
 
+// Workspace: status slot, the per-(b, kv head) range counters right behind it (one clearing
+// memset covers both), then the partials of every key range.
 static size_t decode_ws_bytes(const csa_params* p, int Tq) {
     const Problem P = make_problem(*p, nullptr);
     const DecodePlan d = decode_plan(P, Tq);
-    return kAlign + up(d.qs_bytes) + up(d.part_bytes) + up(d.done_bytes);
+    return kAlign + up(d.done_bytes) + up(d.part_bytes);
 }
 
 size_t csa_decode_workspace_size(const csa_params* p, int Tq) {
@@ -500,22 +509,19 @@ int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_ca
     if ((rc = check_device())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* w = static_cast<uint8_t*>(workspace);
-    if (cudaMemsetAsync(w, 0, 4 * sizeof(int), st) != cudaSuccess) {
-        cudaGetLastError();
-        return CSA_ERR_CUDA;
-    }
     const Problem P = make_problem(*p, reinterpret_cast<int*>(w));
     const DecodePlan d = decode_plan(P, Tq);
-    float* qs = reinterpret_cast<float*>(w + kAlign);
-    float* part = reinterpret_cast<float*>(w + kAlign + up(d.qs_bytes));
-    int* done = reinterpret_cast<int*>(w + kAlign + up(d.qs_bytes) + up(d.part_bytes));
-    if (cudaMemsetAsync(done, 0, d.done_bytes, st) != cudaSuccess) {
+    int* done = reinterpret_cast<int*>(w + kAlign);
+    float* part = reinterpret_cast<float*>(w + kAlign + up(d.done_bytes));
+    CUtensorMap tk, tv;
+    if (!make_map(&tk, k_cache, p->B, p->T, p->Hkv, p->D) || !make_map(&tv, v_cache, p->B, p->T, p->Hkv, p->D))
+        return CSA_ERR_CUDA;
+    // status word and range counters start at zero
+    if (cudaMemsetAsync(w, 0, kAlign + d.done_bytes, st) != cudaSuccess) {
         cudaGetLastError();
         return CSA_ERR_CUDA;
     }
-    if ((rc = timed(kDecodeQ, st, [&] { return launch_decode_q(P, d, q, qs, st); }))) return rc;
-    return timed(kDecodeSplit, st,
-                 [&] { return launch_decode_split(P, d, qs, k_cache, v_cache, part, done, o, lse, st); });
+    return timed(kDecode, st, [&] { return launch_decode(P, d, q, tk, tv, part, done, o, lse, st); });
 }
 
 int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
@@ -596,7 +602,7 @@ int csa_num_kernels(void) { return kNumKernels; }
 const char* csa_kernel_name(int k) {
     static const char* names[kNumKernels] = {"k_prep",          "k_qk_prologue", "k_attn_fwd",
                                              "k_bwd_pre",       "k_attn_bwd",    "k_grad_finalize",
-                                             "k_decode_q",      "k_decode_split"};
+                                             "k_decode"};
     return (k >= 0 && k < kNumKernels) ? names[k] : "";
 }
 
@@ -613,26 +619,17 @@ constexpr size_t kStaticScratchBytes = (size_t)CSA_STATIC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 // Device address of g_static_scratch on the current device.  In host code the array's name
-// is only a host-side stand-in; the real address comes from cudaGetSymbolAddress, looked up
-// once per device (on the first call made with that device current) and cached.
-void* g_static_scratch_addr[64] = {nullptr};
-
+// is only a host-side stand-in; the real address comes from cudaGetSymbolAddress with that
+// device current.  It is looked up on every call (a cheap table lookup once the module is
+// loaded, and it allocates nothing), so a context torn down and re-created by
+// cudaDeviceReset never leaves a stale address behind.
 int static_scratch_address(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
         cudaGetLastError();
         return CSA_ERR_CUDA;
     }
-    if (dev < 0 || dev >= 64) return CSA_ERR_CUDA;
-    if (!g_static_scratch_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return CSA_ERR_CUDA;
-        }
-        g_static_scratch_addr[dev] = p;
-    }
-    *out = g_static_scratch_addr[dev];
+    *out = p;
     return CSA_OK;
 }
 

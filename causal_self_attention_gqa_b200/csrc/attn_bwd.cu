@@ -21,9 +21,10 @@
 // TMEM (512 columns): dV [0,D), dK [128,128+D), S^T [256,384), dP^T [384,512).  P^T is
 // written as packed bf16 over S^T columns (A operand of the dV MMA), dS^T likewise over
 // dP^T columns (A operand of the dK' MMA); dQ' then reuses the dP^T columns.  MMA order per
-// tile: dV(i), S^T(i+1), dK'(i), dQ'(i), then dP^T(i+1) once the drain has read dQ' out of
-// TMEM.  The P/dS warps compute P of tile i+1 (needs S^T only) while dK', dQ' and the drain
-// run, then dS once dP^T arrives.  dS^T also goes to shared memory (128x128 bf16, 128-byte
+// tile: dV(i) and S^T(i+1) as soon as P^T(i) is in TMEM (while the P/dS warps still form
+// dS(i)), then dK'(i), dQ'(i) once dS(i) is complete, then dP^T(i+1) once the drain has read
+// dQ' out of TMEM.  The P/dS warps go from dS(i) straight to P(i+1) (S^T(i+1) is ready by
+// then) while dK', dQ', the drain and dP^T(i+1) run, then dS(i+1) once dP^T arrives.  dS^T also goes to shared memory (128x128 bf16, 128-byte
 // swizzle), where read MN-major it is the A operand of dQ'.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -58,8 +59,9 @@ struct BwdCfg {
     static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;  // 2 x 128 fp32
     static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
     // kv_full, q_full[STAGES], do_full[STAGES], q_empty[STAGES], do_empty[STAGES], s_full,
-    // dp_full, ds_full, ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync, epi_sync[2]
-    static constexpr int NBAR = 1 + 4 * STAGES + 11;
+    // dp_full, ds_full, ds_free, dq_full, dq_empty, acc_full, wg_sync, drain_sync, epi_sync[2],
+    // p_full
+    static constexpr int NBAR = 1 + 4 * STAGES + 12;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -101,7 +103,9 @@ __device__ __forceinline__ void col_bounds(const Problem& P, int b, int j, int& 
     hi = h;
 }
 
-template <int D, bool CAP>
+// CM: soft-cap mode, 0 off, 1 hardware tanh (MUFU), 2 tanh series on the FMA pipe (scores
+// bounded by QK-norm, see cap_series).
+template <int D, int CM>
 __global__ void __launch_bounds__(512, 1)
     k_attn_bwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -129,6 +133,7 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* wg_sync = s_full + 7;     // the P/dS warpgroup's own barrier (bounded, unlike bar.sync)
     uint64_t* drain_sync = s_full + 8;  // the dQ drain warpgroup's own barrier
     uint64_t* epi_sync = s_full + 9;    // [2] each P/dS half's epilogue staging is complete
+    uint64_t* p_full = s_full + 11;     // P^T of the current tile is in TMEM (the dV MMA's A)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     float* lse_s = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -166,6 +171,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
+        mbar_init(p_full, 8);       // one arrival per P/dS warp
         mbar_init(ds_full, 8);      // one arrival per P/dS warp
         mbar_init(ds_free, 1);
         mbar_init(dq_full, 1);
@@ -259,7 +265,9 @@ __global__ void __launch_bounds__(512, 1)
                 const int s = it % NS;
                 const bool next = it + 1 < nit;
                 const int s1 = (it + 1) % NS, ph1 = ((it + 1) / NS) & 1;
-                if (!(ok = mbar_wait(ds_full, it & 1, abort_flag, P.status))) break;
+                // dV needs only P^T: it (and the next S^T behind it) runs while the P/dS warps
+                // are still forming dS of this tile
+                if (!(ok = mbar_wait(p_full, it & 1, abort_flag, P.status))) break;
                 tc_fence_after();
                 // dV += P^T dO   (A = P^T from TMEM; B = dO, MN-major)
 #pragma unroll
@@ -273,6 +281,8 @@ __global__ void __launch_bounds__(512, 1)
                     tc_fence_after();
                     issue_s(s1);
                 }
+                if (!(ok = mbar_wait(ds_full, it & 1, abort_flag, P.status))) break;
+                tc_fence_after();
                 // dK' += dS^T Q'  (A = dS^T from TMEM, packed over dP^T columns; B = Q', MN-major)
 #pragma unroll
                 for (int ks = 0; ks < kBM / 16; ++ks)
@@ -355,31 +365,43 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) {
                     const float4 l4 = *reinterpret_cast<const float4*>(ls + 32 * c + e);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    float pp[4], pf[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float raw = __uint_as_float(sv[e + u]);
-                        float p, dfac = 1.f;
-                        if constexpr (CAP) {
-                            const float t = tanh_approx(raw * P.cap_in);
-                            p = ex2(fmaf(P.cap_log2, t, -lv[u]));
-                            dfac = 1.0f - t * t;
+                    const float2 r01 = make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1]));
+                    const float2 r23 = make_float2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3]));
+                    const float2 nl01 = make_float2(-l4.x, -l4.y), nl23 = make_float2(-l4.z, -l4.w);
+                    float2 x01, x23, t01, t23;
+                    if constexpr (CM == 0) {
+                        const float2 sl2 = make_float2(P.scale_log2, P.scale_log2);
+                        x01 = ffma2(r01, sl2, nl01);
+                        x23 = ffma2(r23, sl2, nl23);
+                    } else {
+                        const float2 cin = make_float2(P.cap_in, P.cap_in), cl2 = make_float2(P.cap_log2, P.cap_log2);
+                        if constexpr (CM == 1) {
+                            t01 = make_float2(tanh_approx(r01.x * P.cap_in), tanh_approx(r01.y * P.cap_in));
+                            t23 = make_float2(tanh_approx(r23.x * P.cap_in), tanh_approx(r23.y * P.cap_in));
                         } else {
-                            p = ex2(fmaf(raw, P.scale_log2, -lv[u]));
+                            t01 = tanh_series2(fmul2(r01, cin));
+                            t23 = tanh_series2(fmul2(r23, cin));
                         }
-                        if (!full) {
+                        x01 = ffma2(t01, cl2, nl01);
+                        x23 = ffma2(t23, cl2, nl23);
+                    }
+                    float pp[4] = {ex2(x01.x), ex2(x01.y), ex2(x23.x), ex2(x23.y)};
+                    if (!full) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
                             const int q = q0 + 32 * c + e + u;
-                            if (q < lo || q > hi) p = 0.f;
+                            if (q < lo || q > hi) pp[u] = 0.f;
                         }
-                        pp[u] = p;
-                        pf[u] = p * dfac;
                     }
                     pk[e / 2] = pack_bf16x2(pp[0], pp[1]);
                     pk[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
-                    if constexpr (CAP) {
-                        pd[cc][e / 2] = pack_bf16x2(pf[0], pf[1]);
-                        pd[cc][e / 2 + 1] = pack_bf16x2(pf[2], pf[3]);
+                    if constexpr (CM != 0) {
+                        // P times the cap's derivative factor 1 - tanh^2
+                        const float2 one = make_float2(1.f, 1.f);
+                        const float2 f01 = fmul2(make_float2(pp[0], pp[1]), ffma2(t01, make_float2(-t01.x, -t01.y), one));
+                        const float2 f23 = fmul2(make_float2(pp[2], pp[3]), ffma2(t23, make_float2(-t23.x, -t23.y), one));
+                        pd[cc][e / 2] = pack_bf16x2(f01.x, f01.y);
+                        pd[cc][e / 2 + 1] = pack_bf16x2(f23.x, f23.y);
                     } else {
                         pd[cc][e / 2] = pk[e / 2];
                         pd[cc][e / 2 + 1] = pk[e / 2 + 1];
@@ -387,6 +409,10 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 tmem_st16(t_s + pt_col(2 * c), pk);  // P^T (bf16) over this half's S^T columns already read
             }
+            // P^T is complete in TMEM: the dV MMA (and the next S^T behind it) may start
+            tmem_st_wait();
+            tc_fence_before();
+            warp_arrive(p_full);
             // dS phase: dP^T of this tile, and the dS buffer free (dQ' of the last tile done)
             ok = mbar_wait(dp_full, it & 1, abort_flag, P.status);
             if (ok && it > 0) ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, P.status);
@@ -612,18 +638,13 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
-template <int D, bool CAP>
+template <int D, int CM>
 static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
                                 const float* lse, const float* delta, float* dq_acc, cudaStream_t st) {
     using C = BwdCfg<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_attn_bwd<D, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(k_attn_bwd<D, CM>), C::SMEM);
+    if (e != cudaSuccess) return e;
     BwdArgs A;
     A.P = P;
     A.lse = lse;
@@ -631,7 +652,7 @@ static cudaError_t launch_bwd_cap(const Problem& P, const CUtensorMap& tq, const
     A.dq_acc = dq_acc;
     A.nkt = (P.T + kBN - 1) / kBN;
     const int grid = A.nkt * P.B * P.Hkv;
-    k_attn_bwd<D, CAP><<<grid, 512, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, tdv, tdk, A);
+    k_attn_bwd<D, CM><<<grid, 512, C::SMEM, st>>>(tq, tk, tv, tdo, tdq, tdv, tdk, A);
     return cudaGetLastError();
 }
 
@@ -639,9 +660,9 @@ template <int D>
 static cudaError_t launch_bwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdq, const CUtensorMap& tdv, const CUtensorMap& tdk,
                                 const float* lse, const float* delta, float* dq_acc, cudaStream_t st) {
-    return (P.softcap > 0.f)
-               ? launch_bwd_cap<D, true>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st)
-               : launch_bwd_cap<D, false>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st);
+    if (P.softcap <= 0.f) return launch_bwd_cap<D, 0>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st);
+    return P.cap_series ? launch_bwd_cap<D, 2>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st)
+                        : launch_bwd_cap<D, 1>(P, tq, tk, tv, tdo, tdq, tdv, tdk, lse, delta, dq_acc, st);
 }
 
 cudaError_t launch_bwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

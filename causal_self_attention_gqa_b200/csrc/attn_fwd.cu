@@ -146,7 +146,9 @@ __device__ __forceinline__ FwdItem decode_item(const FwdArgs& A, int idx) {
     return w;
 }
 
-template <int D, bool CAP>
+// CM: soft-cap mode, 0 off, 1 hardware tanh (MUFU), 2 tanh series on the FMA pipe (scores
+// bounded by QK-norm, see cap_series).
+template <int D, int CM>
 __global__ void __launch_bounds__(384, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -373,9 +375,19 @@ __global__ void __launch_bounds__(384, 1)
                 // logits in log2 units: with the cap x = c log2(e) tanh(s / c) (computed here);
                 // without it x = raw * scale_log2, so the max and the mask work on the raw
                 // scores and the scale folds into the exponent's FFMA (scale > 0)
-                if constexpr (CAP) {
+                if constexpr (CM == 1) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c) raw[c] = __float_as_uint(capped_log2(__uint_as_float(raw[c]), P));
+                } else if constexpr (CM == 2) {
+                    const float2 cin = make_float2(P.cap_in, P.cap_in), cl2 = make_float2(P.cap_log2, P.cap_log2);
+#pragma unroll
+                    for (int c = 0; c < 128; c += 2) {
+                        const float2 x = fmul2(
+                            tanh_series2(fmul2(make_float2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), cin)),
+                            cl2);
+                        raw[c] = __float_as_uint(x.x);
+                        raw[c + 1] = __float_as_uint(x.y);
+                    }
                 }
                 const bool full = (k0 >= lo) && (k0 + kBN - 1 <= hi);
                 if (!full) {
@@ -392,7 +404,7 @@ __global__ void __launch_bounds__(384, 1)
                     for (int u = 0; u < 4; ++u)
                         mx4[u] = fmax3(mx4[u], __uint_as_float(raw[c + 2 * u]), __uint_as_float(raw[c + 2 * u + 1]));
                 }
-                const float xmul = CAP ? 1.0f : P.scale_log2;
+                const float xmul = CM ? 1.0f : P.scale_log2;
                 const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * xmul;
                 // rescale only when the running max grows by more than 2^8 (exact either way:
                 // O and l always share the same reference max)
@@ -407,7 +419,9 @@ __global__ void __launch_bounds__(384, 1)
                 const float2 xm2 = make_float2(xmul, xmul), nb2 = make_float2(nbase, nbase);
                 float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
                 // p = 2^(x - m): MUFU for most pairs; in tiles with no masked key (warp-uniform)
-                // one pair in four goes to the FMA pipe so both units share the work
+                // one pair in four goes to the FMA pipe so both units share the work (one in
+                // two when tanh takes a MUFU slot too; none when the series tanh already loads
+                // the FMA pipe)
                 auto exp_pass = [&](auto emu_tag) {
                     constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
@@ -419,8 +433,7 @@ __global__ void __launch_bounds__(384, 1)
                                                                 __uint_as_float(raw[32 * c + 2 * e + 1])),
                                                     xm2, nb2);
                             float2 pv;
-                            // with the cap, tanh takes a MUFU slot too: emulate one pair in two
-                            if (kEmu && (CAP ? (e & 1) == 1 : (e & 3) == 3))
+                            if (kEmu && (CM == 1 ? (e & 1) == 1 : (CM == 0 && (e & 3) == 3)))
                                 pv = exp2_fma2(make_float2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f)));
                             else
                                 pv = make_float2(ex2(xv.x), ex2(xv.y));
@@ -514,17 +527,12 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int D, bool CAP>
+template <int D, int CM>
 static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, float* lse, cudaStream_t st) {
     using C = FwdCfg<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_attn_fwd<D, CAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = ensure_dyn_smem(reinterpret_cast<const void*>(k_attn_fwd<D, CM>), C::SMEM);
+    if (e != cudaSuccess) return e;
     FwdArgs A;
     A.P = P;
     A.lse = lse;
@@ -538,15 +546,16 @@ static cudaError_t launch_fwd_cap(const Problem& P, const CUtensorMap& tq, const
         A.items = P.B * P.Hq * A.pairs;
     }
     const int grid = A.items < num_sms() ? A.items : num_sms();
-    k_attn_fwd<D, CAP><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, to, A);
+    k_attn_fwd<D, CM><<<grid, 384, C::SMEM, st>>>(tq, tk, tv, to, A);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_fwd_d(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, float* lse, cudaStream_t st) {
-    return (P.softcap > 0.f) ? launch_fwd_cap<D, true>(P, tq, tk, tv, to, lse, st)
-                             : launch_fwd_cap<D, false>(P, tq, tk, tv, to, lse, st);
+    if (P.softcap <= 0.f) return launch_fwd_cap<D, 0>(P, tq, tk, tv, to, lse, st);
+    return P.cap_series ? launch_fwd_cap<D, 2>(P, tq, tk, tv, to, lse, st)
+                        : launch_fwd_cap<D, 1>(P, tq, tk, tv, to, lse, st);
 }
 
 cudaError_t launch_fwd(const Problem& P, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

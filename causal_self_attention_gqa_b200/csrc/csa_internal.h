@@ -1,7 +1,10 @@
 // csa_internal.h -- definitions shared by the host code and the kernels of libcsa.
 #pragma once
+#include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+
+#include <cuda_runtime.h>
 
 #include "csa.h"
 
@@ -46,13 +49,14 @@ struct Problem {
     float softcap;          // 0 = off
     float cap_in;           // scale / softcap: tanh argument per raw score (cap on)
     float cap_log2;         // softcap * log2(e): capped logit in log2 units per unit of tanh
+    int cap_series;         // 1: every |scale * q'.k' / softcap| <= 1/4 is guaranteed (QK-norm on
+                            // our own prologue's output), so tanh may use its short series
     float scale;            // effective score scale
     float scale_log2;       // scale * log2(e)
     int rope, qk_norm;
     float eps;
     const int32_t* seg_start;  // [B, T] first index of each token's segment, or null
     const int32_t* seg_end;    // [B, T] one past its last index, or null
-    const float2* rope_cs;     // [T, D/2] (cos, sin) of pos * base^(-2d/D), or null
     double rope_log_base;      // ln(base) when RoPE is on
     FastDiv div_hq, div_hkv, div_t, div_tq;  // row -> (token, head), token -> (batch row, position)
     int* status;               // device status word (workspace, or the caller's)
@@ -60,19 +64,35 @@ struct Problem {
                                // zeroed by every call): forward, backward
 };
 
+// RoPE frequencies theta_d = base^(-2d/D), d < D/2, computed on the host in fp64 and passed
+// to the kernels that rotate (by value, as a kernel parameter).
+struct RopeFreq {
+    double theta[64];
+};
+inline RopeFreq rope_freq(int D, double log_base) {
+    RopeFreq F;
+    for (int i = 0; i < 64; ++i) F.theta[i] = (i < D / 2) ? exp((-2.0 * i / D) * log_base) : 0.0;
+    return F;
+}
+
 // Work split of the KV-cache decode (decode.cu): Tq new queries, R = G * Tq rows per
 // (b, kv head), the cache cut into `splits` ranges of keys_per_split keys.
 struct DecodePlan {
     int Tq, R, splits, keys_per_split;
-    size_t qs_bytes, part_bytes, done_bytes;
+    size_t part_bytes, done_bytes;
 };
 
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the CURRENT device, once per
+// (kernel, device): the attribute is per device, so a process that drives several GPUs sets
+// it on each.  Thread-safe.
+cudaError_t ensure_dyn_smem(const void* kernel, int bytes);
+
 // Kernel ids for the timing interface (order = csa_kernel_name()).
 enum KernelId {
-    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecodeQ, kDecodeSplit, kNumKernels
+    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecode, kNumKernels
 };
 
 }  // namespace csa

@@ -10,95 +10,63 @@
 // "Architecture").
 //
 // Decoding reads the whole cache for a handful of queries, so it is bound by HBM bandwidth,
-// not by the tensor cores: the work runs on the CUDA cores, split over the cache.
-//   k_decode_q       q' = RoPE(RMSNorm(q)) * scale for the G * Tq rows of every (b, kv head),
-//                    fp32; the rotation phase is formed and reduced in fp64 (positions reach
-//                    2^20)
-//   k_decode_split   one CTA per (key range, kv head, b): each warp streams 32 keys at a time
-//                    (lane = key for the scores, lane = 4 dimensions for P V), online softmax
-//                    in log2 units; the CTA's partial (m, l, o) goes to the workspace, and the
-//                    last CTA of each (b, kv head) merges them: o = sum 2^(m_s - m) o_s / l
+// not by the tensor cores: the arithmetic runs on the CUDA cores and the kernel is built
+// around keeping the memory system busy.  One launch, k_decode, one CTA per (key range,
+// kv head, b):
+//   * the CTA first forms q' = RoPE(RMSNorm(q)) * scale for the R = G * Tq query rows of its
+//     (b, kv head) in shared memory (fp32; the rotation angle in fp64, positions reach 2^20);
+//   * a producer warp streams the range in 128-key chunks with TMA tile loads (the same
+//     swizzled 128-row boxes as the attention kernels) into a ring of K/V stages, so several
+//     chunks are in flight per CTA at any time;
+//   * four compute warps take 32 keys of each chunk: lane = key for the scores (rows of the
+//     swizzled tile read without bank conflicts), lane = 4 dimensions for P V, online
+//     softmax in log2 units;
+//   * the CTA's partial (m, l, o) goes to the workspace, and the last CTA of each
+//     (b, kv head) to count itself done merges every range: o = sum 2^(m_s - m) o_s / l.
+//     It also resets that counter, so the next call needs no clearing pass.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
 
 #include "csa_internal.h"
 #include "ptx.cuh"
+#include "rowops.cuh"
 
 namespace csa {
 
-constexpr int kDecThreads = 128;  // 4 warps per CTA
-constexpr int kDecKeysPerCta = 128;  // smallest key range per CTA
+constexpr int kDecWarps = 4;                    // compute warps; warp 4 is the TMA producer
+constexpr int kDecThreads = 32 * (kDecWarps + 1);
+constexpr int kDecChunk = 32 * kDecWarps;       // keys per chunk (one 128-row TMA box)
 
-// ------------------------------------------------------------------ q prologue
-// RoPE frequencies base^(-2d/D), d < D/2, computed on the host in fp64.
-struct RopeFreq {
-    double theta[64];
+template <int D, int RMAX>
+struct DecCfg {
+    static constexpr int SW = (D % 64 == 0) ? 128 : 64;  // swizzle span of a tile row (bytes)
+    static constexpr int AE = SW / 2;                     // bf16 elements per swizzle row
+    static constexpr int NA = D / AE;                     // swizzle-atom columns per tile
+    static constexpr int TILE = kDecChunk * D * 2;        // one K (or V) chunk
+    // stages: enough bytes in flight per SM with two CTAs resident where they fit
+    static constexpr int STAGES = (D <= 32) ? 4 : ((D <= 64) ? 3 : 2);
+    static constexpr int OFF_KV = 0;                                   // [STAGES][K tile, V tile]
+    static constexpr int OFF_Q = OFF_KV + STAGES * 2 * TILE;           // q' [RMAX][D] fp32
+    static constexpr int OFF_WO = OFF_Q + RMAX * D * 4;                // [4][RMAX][D] fp32
+    static constexpr int OFF_WML = OFF_WO + kDecWarps * RMAX * D * 4;  // m, l [4][RMAX] each
+    static constexpr int OFF_BAR = OFF_WML + 2 * kDecWarps * RMAX * 4;
+    static constexpr int NBAR = 2 * STAGES;                            // full[S], empty[S]
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                // abort flag, last flag
+    static constexpr int SMEM = OFF_MISC + 16;
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(OFF_BAR % 8 == 0, "barrier alignment");
 };
 
-// One warp per query row (b, i, h); writes qs[b][kvh][r][d], r = (h % G) * Tq + i.
-template <int D>
-__global__ void __launch_bounds__(128) k_decode_q(const __nv_bfloat16* __restrict__ q, float* __restrict__ qs,
-                                                  Problem P, int Tq, const RopeFreq F) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    const int rows = P.B * Tq * P.Hq;
-    if (warp >= rows) return;  // whole warps leave together
-    const int h = warp % P.Hq, i = (warp / P.Hq) % Tq, b = warp / (P.Hq * Tq);
-    const __nv_bfloat16* x = q + ((size_t)(b * Tq + i) * P.Hq + h) * D;
-    constexpr int kPer = D / 32;  // elements per lane: d = lane + 32 t
-    float v[kPer];
-    float ss = 0.f;
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-        v[t] = __bfloat162float(x[lane + 32 * t]);
-        ss += v[t] * v[t];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float r = P.qk_norm ? rsqrtf(ss * (1.0f / D) + P.eps) : 1.0f;
-    __shared__ float row[4][D];
-    float* y = row[threadIdx.x >> 5];
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) y[lane + 32 * t] = v[t] * r;
-    __syncwarp();
-    if (P.rope) {
-        const int pos = P.T - Tq + i;
-        float out[kPer];
-#pragma unroll
-        for (int t = 0; t < kPer; ++t) {
-            const int d = lane + 32 * t, d2 = d % (D / 2);
-            // phase pos * theta in fp64 (it reaches ~1e6 rad), reduced to [-pi, pi] with a
-            // two-part 2 pi (Cody-Waite), then the fp32 sine / cosine of the remainder
-            const double phi = (double)pos * F.theta[d2];
-            const double k = rint(phi * 0.15915494309189535);  // 1 / (2 pi)
-            const double red = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, phi));
-            float sn, cs;
-            sincosf((float)red, &sn, &cs);
-            const float a = y[d2], bb = y[d2 + D / 2];
-            out[t] = (d < D / 2) ? a * cs - bb * sn : bb * cs + a * sn;
-        }
-        __syncwarp();
-#pragma unroll
-        for (int t = 0; t < kPer; ++t) y[lane + 32 * t] = out[t];
-        __syncwarp();
-    }
-    const int G = P.G, kvh = h / G, rr = (h % G) * Tq + i, R = G * Tq;
-    float* dst = qs + (((size_t)b * P.Hkv + kvh) * R + rr) * D;
-#pragma unroll
-    for (int t = 0; t < kPer; ++t) dst[lane + 32 * t] = y[lane + 32 * t] * P.scale;
-}
-
-// ------------------------------------------------------------------ split over the cache
 struct DecArgs {
     Problem P;
-    int Tq, R, splits, keys_per_split;
-    const float* qs;               // [B, Hkv, R, D] q' * scale
-    const __nv_bfloat16* kc;       // [B, Tk, Hkv, D]
-    const __nv_bfloat16* vc;       // [B, Tk, Hkv, D]
-    float* part;                   // [B, Hkv, splits, R, D + 2]: o (unnormalised), m, l
-    int* done;                     // [B, Hkv] key ranges finished (zeroed by the call)
-    __nv_bfloat16* o;              // [B, Tq, Hq, D]
-    float* lse;                    // [B, Hq, Tq]
+    int Tq, R, splits, keys_per_split;  // keys_per_split: a multiple of kDecChunk
+    const __nv_bfloat16* q;             // [B, Tq, Hq, D] raw
+    float* part;                        // [B, Hkv, splits, R, D + 2]: o (unnormalised), m, l
+    int* done;                          // [B, Hkv] key ranges finished (zero between calls)
+    __nv_bfloat16* o;                   // [B, Tq, Hq, D]
+    float* lse;                         // [B, Hq, Tq]
 };
 
 // o and LSE of one (b, kv head) from the partials of all its key ranges:
@@ -139,133 +107,219 @@ __device__ __forceinline__ void dec_bounds(const Problem& P, int Tq, int r, int&
     }
 }
 
+// Byte offset of element d of row r in a swizzled 128-row tile (atoms of 128 rows x SW bytes,
+// 16-byte chunk j of row r stored at chunk j ^ x(r), the pattern the TMA box writes).
+template <int SW>
+__device__ __forceinline__ uint32_t swz_off(int r, int d) {
+    constexpr int AE = SW / 2;
+    const int a = d / AE, j = (d % AE) / 8, w = d % 8;
+    const int x = (SW == 128) ? (r & 7) : ((r >> 1) & 3);
+    return (uint32_t)(a * (kDecChunk * SW) + r * SW + ((j ^ x) * 16) + w * 2);
+}
+
 template <int D, int RMAX, bool CAP>
-__global__ void __launch_bounds__(kDecThreads, RMAX >= 16 ? 2 : 4) k_decode_split(const DecArgs A) {
+__global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ CUtensorMap tm_k,
+                                                       const __grid_constant__ CUtensorMap tm_v, const DecArgs A,
+                                                       const RopeFreq F) {
+    using C = DecCfg<D, RMAX>;
+    extern __shared__ __align__(1024) uint8_t smem[];
     const Problem& P = A.P;
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int R = A.R;
-    __shared__ float qsh[RMAX][D];
-    __shared__ float wm[4][RMAX], wl[4][RMAX];
-    __shared__ float wo[4][RMAX][D];
-    const float* qsrc = A.qs + ((size_t)b * P.Hkv + kvh) * R * D;
-    for (int e = threadIdx.x; e < RMAX * D; e += kDecThreads) qsh[e / D][e % D] = (e / D < R) ? qsrc[e] : 0.f;
-    __syncthreads();
+    float(*qsh)[D] = reinterpret_cast<float(*)[D]>(smem + C::OFF_Q);
+    float(*wo)[RMAX][D] = reinterpret_cast<float(*)[RMAX][D]>(smem + C::OFF_WO);
+    float(*wm)[RMAX] = reinterpret_cast<float(*)[RMAX]>(smem + C::OFF_WML);
+    float(*wl)[RMAX] = reinterpret_cast<float(*)[RMAX]>(smem + C::OFF_WML + kDecWarps * RMAX * 4);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + C::STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+    int* last = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
-    const float kLog2e = 1.4426950408889634f;
-    float m[RMAX], l[RMAX], acc[RMAX][4];
-#pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-        m[r] = -INFINITY;
-        l[r] = 0.f;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc[r][t] = 0.f;
+    // the swizzled tiles need a 1024-byte aligned base; the condition is uniform over the CTA
+    if ((smem_u32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(P.status, 0, CSA_ERR_LAUNCH);
+        return;
     }
     const int k_begin = split * A.keys_per_split;
     const int k_end = min(P.T, k_begin + A.keys_per_split);
-    const size_t row_stride = (size_t)P.Hkv * D;  // elements between consecutive cache rows
-    const __nv_bfloat16* kbase = A.kc + ((size_t)b * P.T * P.Hkv + kvh) * D;
-    const __nv_bfloat16* vbase = A.vc + ((size_t)b * P.T * P.Hkv + kvh) * D;
-    const bool pv_lane = 4 * lane < D;  // lane owns dimensions [4 lane, 4 lane + 4) in P V
+    const int nchunks = k_end > k_begin ? (k_end - k_begin + kDecChunk - 1) / kDecChunk : 0;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kDecWarps);  // one arrival per compute warp
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
 
-    // warps take interleaved chunks of 32 keys
-    for (int k0 = k_begin + 32 * warp; k0 < k_end; k0 += 32 * 4) {
-        const int key = k0 + lane;
-        const bool kin = key < k_end;
-        // scores of this lane's key against every row (q' rows broadcast from shared memory)
-        float s[RMAX];
+    if (warp == kDecWarps) {
+        // ================= producer: K and V chunks of the range into the stage ring
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % C::STAGES;
+                if (c >= C::STAGES && !mbar_wait(&empty[s], ((c / C::STAGES) - 1) & 1, abort_flag, P.status)) break;
+                const int k0 = k_begin + c * kDecChunk;
+                uint8_t* kt = smem + C::OFF_KV + s * 2 * C::TILE;
+                mbar_arrive_expect_tx(&full[s], 2 * C::TILE);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_k, &full[s], kt + a * kDecChunk * C::SW, a * C::AE, kvh, k0, b);
+                for (int a = 0; a < C::NA; ++a)
+                    tma_load_4d(&tm_v, &full[s], kt + C::TILE + a * kDecChunk * C::SW, a * C::AE, kvh, k0, b);
+            }
+        }
+    } else {
+        // ================= q' of the R rows: one warp per row (rows w, w + 4, ...)
+        constexpr int kPer = D / 32;  // elements per lane: d = lane + 32 t
+        for (int r = warp; r < RMAX; r += kDecWarps) {
+            if (r >= R) {
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) s[r] = 0.f;
-        if (kin) {
-            const uint4* kr = reinterpret_cast<const uint4*>(kbase + (size_t)key * row_stride);
+                for (int t = 0; t < kPer; ++t) qsh[r][lane + 32 * t] = 0.f;
+                continue;
+            }
+            const int i = r % A.Tq, h = kvh * P.G + r / A.Tq;
+            const __nv_bfloat16* x = A.q + ((size_t)(b * A.Tq + i) * P.Hq + h) * D;
+            float v[kPer];
+            float ss = 0.f;
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) {
+                v[t] = __bfloat162float(x[lane + 32 * t]);
+                ss += v[t] * v[t];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float rn = P.qk_norm ? rsqrtf(ss * (1.0f / D) + P.eps) : 1.0f;
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) qsh[r][lane + 32 * t] = v[t] * rn;
+            __syncwarp();
+            float out[kPer];
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) {
+                const int d = lane + 32 * t, d2 = d % (D / 2);
+                float y = qsh[r][d];
+                if (P.rope) {
+                    const float2 ang = rope_angle(P.T - A.Tq + i, F.theta[d2]);
+                    const float a = qsh[r][d2], bb = qsh[r][d2 + D / 2];
+                    y = (d < D / 2) ? a * ang.x - bb * ang.y : bb * ang.x + a * ang.y;
+                }
+                out[t] = y * P.scale;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) qsh[r][lane + 32 * t] = out[t];
+        }
+        // the four compute warps share the q' rows
+        named_bar_sync(1, 32 * kDecWarps);
+
+        const float kLog2e = 1.4426950408889634f;
+        float m[RMAX], l[RMAX], acc[RMAX][4];
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            m[r] = -INFINITY;
+            l[r] = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) acc[r][t] = 0.f;
+        }
+        const bool pv_lane = 4 * lane < D;  // lane owns dimensions [4 lane, 4 lane + 4) in P V
+        const int row = 32 * warp + lane;    // this lane's key row in every chunk (scores)
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % C::STAGES;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (c / C::STAGES) & 1, abort_flag, P.status))) break;
+            const uint8_t* kt = smem + C::OFF_KV + s * 2 * C::TILE;
+            const uint8_t* vt = kt + C::TILE;
+            const int k0 = k_begin + c * kDecChunk + 32 * warp;  // this warp's first key
+            const int key = k0 + lane;
+            const bool kin = key < k_end;
+            // scores of this lane's key against every row (q' rows broadcast from shared memory)
+            float sc[RMAX];
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) sc[r] = 0.f;
 #pragma unroll 4
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 u = kr[c];
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            for (int d8 = 0; d8 < D; d8 += 8) {
+                const uint4 u = *reinterpret_cast<const uint4*>(kt + swz_off<C::SW>(row, d8));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
                 float kf[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    kf[2 * e] = __uint_as_float(w[e] << 16);
-                    kf[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                    kf[2 * e] = __uint_as_float(wv[e] << 16);
+                    kf[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
                 }
 #pragma unroll
                 for (int r = 0; r < RMAX; ++r)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s[r] = fmaf(qsh[r][8 * c + e], kf[e], s[r]);
+                    for (int e = 0; e < 8; ++e) sc[r] = fmaf(qsh[r][d8 + e], kf[e], sc[r]);
             }
-        }
-        // logits in log2 units, masked to -inf
-        float x[RMAX];
+            // logits in log2 units, masked to -inf
+            float x[RMAX];
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-            int lo, hi;
-            dec_bounds(P, A.Tq, r, lo, hi);
-            const float v = CAP ? P.cap_log2 * tanh_approx(s[r] * (1.0f / P.softcap)) : s[r] * kLog2e;
-            x[r] = (r < R && kin && key >= lo && key <= hi) ? v : -INFINITY;
-        }
-        // online softmax per row over this chunk
-        float p[RMAX];
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-            float cm = x[r];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
-            const float mn = fmaxf(m[r], cm);
-            const float alpha = (m[r] == -INFINITY) ? 0.f : ex2(m[r] - mn);
-            p[r] = (x[r] == -INFINITY) ? 0.f : ex2(x[r] - mn);
-            float ps = p[r];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-            if (mn != -INFINITY) {
-                l[r] = l[r] * alpha + ps;
-#pragma unroll
-                for (int t = 0; t < 4; ++t) acc[r][t] *= alpha;
-                m[r] = mn;
+            for (int r = 0; r < RMAX; ++r) {
+                int lo, hi;
+                dec_bounds(P, A.Tq, r, lo, hi);
+                const float v = CAP ? P.cap_log2 * tanh_approx(sc[r] * (1.0f / P.softcap)) : sc[r] * kLog2e;
+                x[r] = (r < R && kin && key >= lo && key <= hi) ? v : -INFINITY;
             }
-        }
-        // P V: key kk's probabilities broadcast from lane kk; lane owns 4 consecutive dims.
-        // Value rows are fetched 8 keys at a time, so their loads are in flight together.
-        const int nk = min(32, k_end - k0);
-        for (int k8 = 0; k8 < nk; k8 += 8) {
-            uint2 vu[8];
+            // online softmax per row over this warp's 32 keys
+            float p[RMAX];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                vu[u] = make_uint2(0u, 0u);
-                if (pv_lane && k8 + u < nk)
-                    vu[u] = *reinterpret_cast<const uint2*>(vbase + (size_t)(k0 + k8 + u) * row_stride + 4 * lane);
+            for (int r = 0; r < RMAX; ++r) {
+                float cm = x[r];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+                const float mn = fmaxf(m[r], cm);
+                const float alpha = (m[r] == -INFINITY) ? 0.f : ex2(m[r] - mn);
+                p[r] = (x[r] == -INFINITY) ? 0.f : ex2(x[r] - mn);
+                float ps = p[r];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+                if (mn != -INFINITY) {
+                    l[r] = l[r] * alpha + ps;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) acc[r][t] *= alpha;
+                    m[r] = mn;
+                }
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float vf[4] = {__uint_as_float(vu[u].x << 16), __uint_as_float(vu[u].x & 0xffff0000u),
-                                     __uint_as_float(vu[u].y << 16), __uint_as_float(vu[u].y & 0xffff0000u)};
+            // P V: key kk's probabilities broadcast from lane kk; lane owns 4 consecutive dims
+            const int nk = max(0, min(32, k_end - k0));
+#pragma unroll 4
+            for (int kk = 0; kk < nk; ++kk) {
+                uint2 vu = make_uint2(0u, 0u);
+                if (pv_lane) vu = *reinterpret_cast<const uint2*>(vt + swz_off<C::SW>(32 * warp + kk, 4 * lane));
+                const float vf[4] = {__uint_as_float(vu.x << 16), __uint_as_float(vu.x & 0xffff0000u),
+                                     __uint_as_float(vu.y << 16), __uint_as_float(vu.y & 0xffff0000u)};
 #pragma unroll
                 for (int r = 0; r < RMAX; ++r) {
-                    const float pk = __shfl_sync(0xffffffffu, p[r], (k8 + u) & 31);
+                    const float pk = __shfl_sync(0xffffffffu, p[r], kk);
 #pragma unroll
                     for (int t = 0; t < 4; ++t) acc[r][t] = fmaf(pk, vf[t], acc[r][t]);
                 }
             }
+            warp_arrive(&empty[s]);  // this warp is done with the stage
         }
-    }
-    // merge the four warps, then the CTA's partial goes to the workspace
+        // this warp's partial to shared memory
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-        if (lane == 0) {
-            wm[warp][r] = m[r];
-            wl[warp][r] = l[r];
+        for (int r = 0; r < RMAX; ++r) {
+            if (lane == 0) {
+                wm[warp][r] = m[r];
+                wl[warp][r] = l[r];
+            }
+            if (pv_lane)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) wo[warp][r][4 * lane + t] = acc[r][t];
         }
-        if (pv_lane)
-#pragma unroll
-            for (int t = 0; t < 4; ++t) wo[warp][r][4 * lane + t] = acc[r][t];
     }
     __syncthreads();
+    if (*abort_flag) return;  // a bounded wait ran out: the status word says so, nothing merges
+    // merge the four warps; the CTA's partial goes to the workspace
     float* dst = A.part + ((((size_t)b * P.Hkv + kvh) * A.splits + split) * R) * (D + 2);
-    for (int e = threadIdx.x; e < R * D; e += kDecThreads) {
+    for (int e = threadIdx.x; e < R * D; e += blockDim.x) {
         const int r = e / D, d = e % D;
         float mm = -INFINITY;
-        for (int w = 0; w < 4; ++w) mm = fmaxf(mm, wm[w][r]);
+        for (int w = 0; w < kDecWarps; ++w) mm = fmaxf(mm, wm[w][r]);
         float o = 0.f, ll = 0.f;
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kDecWarps; ++w) {
             const float f = (wm[w][r] == -INFINITY) ? 0.f : ex2(wm[w][r] - mm);
             o += f * wo[w][r][d];
             ll += f * wl[w][r];
@@ -277,27 +331,29 @@ __global__ void __launch_bounds__(kDecThreads, RMAX >= 16 ? 2 : 4) k_decode_spli
         }
     }
     // the last CTA of this (b, kv head) to finish merges every key range (no waiting: the
-    // others have published their partials before counting themselves done)
+    // others have published their partials before counting themselves done), then resets
+    // the counter for the next call
     __threadfence();
     __syncthreads();
-    __shared__ int last;
-    if (threadIdx.x == 0) last = (atomicAdd(&A.done[b * P.Hkv + kvh], 1) == A.splits - 1) ? 1 : 0;
+    int* cnt = &A.done[b * P.Hkv + kvh];
+    if (threadIdx.x == 0) *last = (atomicAdd(cnt, 1) == A.splits - 1) ? 1 : 0;
     __syncthreads();
-    if (!last) return;
+    if (!*last) return;
     __threadfence();
     merge_partials<D>(A, b, kvh);
+    if (threadIdx.x == 0) *cnt = 0;
 }
 
 // ------------------------------------------------------------------ host side
-// Key ranges for `resident` CTAs per SM: one wave of the grid, at least 128 keys per range.
-// The workspace is sized for resident = 8, the most any launch uses.
+// Key ranges (multiples of the 128-key chunk) for `resident` CTAs per SM: one wave of the
+// grid.  The workspace is sized for resident = 8, more than any launch uses.
 static void split_keys(const Problem& P, int resident, int& splits, int& keys_per_split) {
     const int ctas = P.B * P.Hkv;
     int s = ctas > 0 ? resident * num_sms() / ctas : 1;
-    const int max_s = (P.T + kDecKeysPerCta - 1) / kDecKeysPerCta;
+    const int max_s = (P.T + kDecChunk - 1) / kDecChunk;
     s = s < 1 ? 1 : (s > max_s ? max_s : s);
     const int kps = (P.T + s - 1) / s;
-    keys_per_split = (kps + 31) / 32 * 32;
+    keys_per_split = (kps + kDecChunk - 1) / kDecChunk * kDecChunk;
     splits = (P.T + keys_per_split - 1) / keys_per_split;
 }
 
@@ -306,84 +362,60 @@ DecodePlan decode_plan(const Problem& P, int Tq) {
     d.Tq = Tq;
     d.R = P.G * Tq;
     split_keys(P, 8, d.splits, d.keys_per_split);
-    d.qs_bytes = (size_t)P.B * P.Hkv * d.R * P.D * sizeof(float);
     d.part_bytes = (size_t)P.B * P.Hkv * d.splits * d.R * (P.D + 2) * sizeof(float);
     d.done_bytes = (size_t)P.B * P.Hkv * sizeof(int);
     return d;
 }
 
-static DecArgs dec_args(const Problem& P, const DecodePlan& d, const float* qs, const void* kc, const void* vc,
-                        float* part, int* done, void* o, float* lse) {
+template <int D, int RMAX, bool CAP>
+static cudaError_t launch_dec(DecArgs A, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+    using C = DecCfg<D, RMAX>;
+    const void* fn = reinterpret_cast<const void*>(k_decode<D, RMAX, CAP>);
+    cudaError_t e = ensure_dyn_smem(fn, C::SMEM);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode<D, RMAX, CAP>, kDecThreads, C::SMEM) !=
+            cudaSuccess ||
+        n < 1) {
+        cudaGetLastError();
+        n = 1;
+    }
+    split_keys(A.P, n < 8 ? n : 8, A.splits, A.keys_per_split);
+    const RopeFreq F = rope_freq(D, A.P.rope_log_base);
+    dim3 grid(A.splits, A.P.Hkv, A.P.B);
+    k_decode<D, RMAX, CAP><<<grid, kDecThreads, C::SMEM, st>>>(tk, tv, A, F);
+    return cudaGetLastError();
+}
+
+template <int D, bool CAP>
+static cudaError_t launch_dec_r(const DecArgs& A, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+    if (A.R <= 2) return launch_dec<D, 2, CAP>(A, tk, tv, st);
+    if (A.R <= 4) return launch_dec<D, 4, CAP>(A, tk, tv, st);
+    if (A.R <= 8) return launch_dec<D, 8, CAP>(A, tk, tv, st);
+    return launch_dec<D, 16, CAP>(A, tk, tv, st);
+}
+
+cudaError_t launch_decode(const Problem& P, const DecodePlan& d, const void* q, const CUtensorMap& tk,
+                          const CUtensorMap& tv, float* part, int* done, void* o, float* lse, cudaStream_t st) {
     DecArgs A;
     A.P = P;
     A.Tq = d.Tq;
     A.R = d.R;
     A.splits = d.splits;
     A.keys_per_split = d.keys_per_split;
-    A.qs = qs;
-    A.kc = static_cast<const __nv_bfloat16*>(kc);
-    A.vc = static_cast<const __nv_bfloat16*>(vc);
+    A.q = static_cast<const __nv_bfloat16*>(q);
     A.part = part;
     A.done = done;
     A.o = static_cast<__nv_bfloat16*>(o);
     A.lse = lse;
-    return A;
-}
-
-// The grid is one wave: as many key ranges as the SMs hold CTAs of this instance at once
-// (never more than the workspace was sized for).
-template <int D, int RMAX, bool CAP>
-static cudaError_t launch_split(DecArgs A, cudaStream_t st) {
-    static int resident = 0;
-    if (!resident) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_split<D, RMAX, CAP>, kDecThreads, 0) !=
-                cudaSuccess ||
-            n < 1) {
-            cudaGetLastError();
-            n = 4;
-        }
-        resident = n < 8 ? n : 8;
+#define CALL(D_) ((P.softcap > 0.f) ? launch_dec_r<D_, true>(A, tk, tv, st) : launch_dec_r<D_, false>(A, tk, tv, st))
+    switch (P.D) {
+        case 32: return CALL(32);
+        case 64: return CALL(64);
+        case 96: return CALL(96);
+        case 128: return CALL(128);
+        default: return cudaErrorInvalidValue;
     }
-    split_keys(A.P, resident, A.splits, A.keys_per_split);
-    dim3 grid(A.splits, A.P.Hkv, A.P.B);
-    k_decode_split<D, RMAX, CAP><<<grid, kDecThreads, 0, st>>>(A);
-    return cudaGetLastError();
-}
-
-template <int D, bool CAP>
-static cudaError_t launch_split_r(const DecArgs& A, cudaStream_t st) {
-    if (A.R <= 2) return launch_split<D, 2, CAP>(A, st);
-    if (A.R <= 4) return launch_split<D, 4, CAP>(A, st);
-    if (A.R <= 8) return launch_split<D, 8, CAP>(A, st);
-    return launch_split<D, 16, CAP>(A, st);
-}
-
-#define CSA_DEC_DISPATCH(CALL)                  \
-    switch (P.D) {                              \
-        case 32: return CALL(32);               \
-        case 64: return CALL(64);               \
-        case 96: return CALL(96);               \
-        case 128: return CALL(128);             \
-        default: return cudaErrorInvalidValue;  \
-    }
-
-cudaError_t launch_decode_q(const Problem& P, const DecodePlan& d, const void* q, float* qs, cudaStream_t st) {
-    const int rows = P.B * d.Tq * P.Hq;
-    const int blocks = (rows + 3) / 4;
-    RopeFreq F;
-    for (int i = 0; i < P.D / 2; ++i) F.theta[i] = P.rope ? exp((-2.0 * i / P.D) * P.rope_log_base) : 0.0;
-#define CALL(D_)                                                                                              \
-    (k_decode_q<D_><<<blocks, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), qs, P, d.Tq, F), cudaGetLastError())
-    CSA_DEC_DISPATCH(CALL)
-#undef CALL
-}
-
-cudaError_t launch_decode_split(const Problem& P, const DecodePlan& d, const float* qs, const void* kc,
-                                const void* vc, float* part, int* done, void* o, float* lse, cudaStream_t st) {
-    const DecArgs A = dec_args(P, d, qs, kc, vc, part, done, o, lse);
-#define CALL(D_) ((P.softcap > 0.f) ? launch_split_r<D_, true>(A, st) : launch_split_r<D_, false>(A, st))
-    CSA_DEC_DISPATCH(CALL)
 #undef CALL
 }
 

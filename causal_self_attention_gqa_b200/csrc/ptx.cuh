@@ -319,6 +319,20 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
                        __int_as_float(__float_as_int(t.y) * 8388608 + __float_as_int(p.y)));
 }
 
+// tanh(u) for |u| <= 1/4 on the FMA pipe, two values per instruction: the Maclaurin series
+// of tanh through u^7, u (1 + u^2 (-1/3 + u^2 (2/15 - (17/315) u^2))).  On that range the
+// series alternates with shrinking terms, so the truncation error is below the first
+// omitted term, (62/2835) |u|^9 (8.3e-8 at |u| = 1/4, 3.4e-7 relative), plus float rounding:
+// far below the hardware tanh.approx (about 2^-11 relative).  The caller guarantees the range
+// (QK-norm bounds every score; see the cap_series flag on the host).
+__device__ __forceinline__ float2 tanh_series2(float2 u) {
+    const float2 u2 = fmul2(u, u);
+    float2 p = ffma2(u2, make_float2(-5.3968254e-2f, -5.3968254e-2f), make_float2(1.3333334e-1f, 1.3333334e-1f));
+    p = ffma2(p, u2, make_float2(-3.3333334e-1f, -3.3333334e-1f));
+    p = ffma2(p, u2, make_float2(1.0f, 1.0f));
+    return fmul2(u, p);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     // cvt packs its first source into the upper half

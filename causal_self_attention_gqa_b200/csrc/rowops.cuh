@@ -1,8 +1,12 @@
 // rowops.cuh -- small per-row helpers shared by the row kernels and the attention
-// kernels' epilogues: bf16 vector loads/stores, lane-group sums, transposed RoPE.
+// kernels' epilogues: bf16 vector loads/stores, lane-group sums, the RoPE rotation angle,
+// transposed RoPE.
 #pragma once
 #include <cuda_bf16.h>
+#include <math.h>
 #include <stdint.h>
+
+#include "csa_internal.h"
 
 namespace csa {
 
@@ -46,6 +50,18 @@ __device__ __forceinline__ float group_sum(float v) {
 #pragma unroll
     for (int o = GS / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, GS);
     return v;
+}
+// (cos phi, sin phi) of the RoPE angle phi = pos * theta (theta = base^(-2d/D) from the
+// host, fp64).  phi reaches ~1e6 rad at the longest sequences, so it is formed and reduced
+// to [-pi, pi] in fp64 (Cody-Waite, 2 pi split into its nearest double and the remainder),
+// and only the remainder goes to the fp32 sine and cosine.
+__device__ __forceinline__ float2 rope_angle(int pos, double theta) {
+    const double phi = (double)pos * theta;
+    const double k = rint(phi * 0.15915494309189535);  // 1 / (2 pi)
+    const double red = fma(-k, 2.4492935982947064e-16, fma(-k, 6.283185307179586, phi));
+    float sn, cs;
+    sincosf((float)red, &sn, &cs);
+    return make_float2(cs, sn);
 }
 // Transpose of the rotate-half rotation by phi (i.e. rotation by -phi) applied to a
 // gradient pair (g_a at d, g_b at d + D/2); cs = (cos phi, sin phi).

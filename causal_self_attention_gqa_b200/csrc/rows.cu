@@ -1,18 +1,20 @@
 // rows.cu -- the HBM-bound row kernels around the two attention kernels:
-//   k_prep         segment bounds of every token (maximal runs of equal segment_ids) and the
-//                  RoPE (cos, sin) table for positions 0..T-1, computed in fp64
+//   k_prep         segment bounds of every token (maximal runs of equal segment_ids); only
+//                  launched when segment_ids are given
 //   k_qk_prologue  q' = RoPE(RMSNorm(q)), k' = RoPE(RMSNorm(k)) -> bf16 copies in the workspace
 //   k_bwd_pre      delta_i = sum_d dO_id O_id per (b, h, i) and a zeroed fp32 dQ accumulator
 //   k_grad_finalize dq (and dk when QK-norm or RoPE is on) = RMSNorm^T(RoPE^T(scale * acc))
 //                  -> bf16, from the fp32 dQ' accumulator and the raw dK' sums
+// The RoPE angle of position p and frequency theta_d = base^(-2d/D) is formed in the kernels
+// (fp64 phase, reduced, fp32 sine / cosine: rope_angle), once per token and frequency.
 //
 // The norm is the parameter-free RMSNorm and the rotation the rotate-half RoPE of the
 // nanogpt-jax-181m model card ("Architecture"); positions restart at each packed segment
 // (same section, "RoPE frequencies are computed from packed segment positions").
 //
-// Row kernels give each [.., D] row an aligned group of lanes; a lane owns whole rotation
-// pairs (d, d + D/2), so a rotation never crosses lanes.  The finalize uses 16-lane groups
-// with 4 pairs per lane (it holds twice the data per pair, and 16-byte lanes cost it occupancy).
+// The prologue and the finalize give each token an aligned group of lanes that walks over
+// the token's heads; a lane owns whole rotation pairs (d, d + D/2), so a rotation never
+// crosses lanes.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -21,7 +23,7 @@
 
 namespace csa {
 
-// ------------------------------------------------------------------ segments + RoPE table
+// ------------------------------------------------------------------ segment bounds
 template <bool kMax>
 __device__ __forceinline__ int block_scan_1024(int v, int* sh) {
     // inclusive scan (max or min) across the 1024 threads of the block, in thread order
@@ -48,127 +50,133 @@ __device__ __forceinline__ int block_scan_1024(int v, int* sh) {
     return v;
 }
 
-__global__ void __launch_bounds__(1024) k_prep(int B, int T, const int32_t* __restrict__ ids,
-                                               int32_t* __restrict__ seg_start, int32_t* __restrict__ seg_end,
-                                               float2* __restrict__ rope_cs, int half, double log_base) {
+// One block per batch row: seg_start[t] = first index of t's maximal run of equal ids (a
+// running max of run-start indices), seg_end[t] = one past its last index (a running min,
+// from the right, of run ends).
+__global__ void __launch_bounds__(1024) k_prep(int T, const int32_t* __restrict__ ids, int32_t* __restrict__ seg_start,
+                                               int32_t* __restrict__ seg_end) {
     __shared__ int sh[32];
-    const int seg_blocks = ids ? B : 0;
-    if ((int)blockIdx.x < seg_blocks) {
-        const int b = blockIdx.x;
-        const int32_t* id = ids + (size_t)b * T;
-        int carry = 0;
-        for (int base = 0; base < T; base += 1024) {  // start: running max of run-start indices
-            const int t = base + threadIdx.x;
-            int v = -1;
-            if (t < T) v = (t == 0 || id[t] != id[t - 1]) ? t : -1;
-            v = block_scan_1024<true>(v, sh);
-            v = max(v, carry);
-            if (t < T) seg_start[(size_t)b * T + t] = v;
-            if (threadIdx.x == 1023) sh[0] = v;
-            __syncthreads();
-            carry = sh[0];
-            __syncthreads();
-        }
-        carry = T;
-        for (int top = T - 1; top >= 0; top -= 1024) {  // end: running min (from the right) of run ends
-            const int t = top - (int)threadIdx.x;
-            int v = T;
-            if (t >= 0) v = (t == T - 1 || id[t] != id[t + 1]) ? t + 1 : T;
-            v = block_scan_1024<false>(v, sh);
-            v = min(v, carry);
-            if (t >= 0) seg_end[(size_t)b * T + t] = v;
-            if (threadIdx.x == 1023) sh[0] = v;
-            __syncthreads();
-            carry = sh[0];
-            __syncthreads();
-        }
-        return;
+    const int b = blockIdx.x;
+    const int32_t* id = ids + (size_t)b * T;
+    int carry = 0;
+    for (int base = 0; base < T; base += 1024) {
+        const int t = base + threadIdx.x;
+        int v = -1;
+        if (t < T) v = (t == 0 || id[t] != id[t - 1]) ? t : -1;
+        v = block_scan_1024<true>(v, sh);
+        v = max(v, carry);
+        if (t < T) seg_start[(size_t)b * T + t] = v;
+        if (threadIdx.x == 1023) sh[0] = v;
+        __syncthreads();
+        carry = sh[0];
+        __syncthreads();
     }
-    if (!rope_cs) return;
-    const uint32_t idx = (blockIdx.x - seg_blocks) * blockDim.x + threadIdx.x;  // T * half < 2^27
-    if (idx >= (uint32_t)T * half) return;
-    const int t = (int)(idx / half), d = (int)(idx - (uint32_t)t * half);
-    const double theta = exp((-2.0 * d / (2.0 * half)) * log_base);  // base^(-2d/D)
-    double s, c;
-    sincos((double)t * theta, &s, &c);
-    rope_cs[idx] = make_float2((float)c, (float)s);
+    carry = T;
+    for (int top = T - 1; top >= 0; top -= 1024) {
+        const int t = top - (int)threadIdx.x;
+        int v = T;
+        if (t >= 0) v = (t == T - 1 || id[t] != id[t + 1]) ? t + 1 : T;
+        v = block_scan_1024<false>(v, sh);
+        v = min(v, carry);
+        if (t >= 0) seg_end[(size_t)b * T + t] = v;
+        if (threadIdx.x == 1023) sh[0] = v;
+        __syncthreads();
+        carry = sh[0];
+        __syncthreads();
+    }
 }
 
 // ------------------------------------------------------------------ q/k prologue
-// Row geometry of the prologue: a lane owns the 8 rotation pairs
-// (d, d + D/2) for d in [8g, 8g + 8), so its loads and stores are 16 bytes wide; the D/16
-// lanes of a row form an aligned group of GS lanes (a power of two; D = 96 leaves 2 of 8 idle).
+// A group of GS lanes owns one token (b, t) and walks over all of its query heads, then its
+// key heads (4 head rows in flight per lane).  A lane owns the 8 rotation pairs
+// (d, d + D/2) for d in [8g, 8g + 8): its loads and stores are 16 bytes wide, and it forms the
+// RoPE angle of those 8 frequencies once for the token, whatever the number of heads.  The
+// D/16 active lanes of a token form an aligned group of GS lanes (a power of two; D = 96
+// leaves 2 of 8 idle).
 template <int D>
-struct RowGeom {
+struct TokGeom {
     static constexpr int LPR = D / 16;
     static constexpr int GS = (LPR <= 2) ? 2 : (LPR <= 4 ? 4 : 8);
-    static constexpr int ROWS = 256 / GS;  // rows per 256-thread block
+    static constexpr int TOK = 256 / GS;  // tokens per 256-thread block
 };
+
+// Normalises and rotates H head rows of one token: x, y point at the token's first head.
+template <int D>
+__device__ __forceinline__ void prologue_heads(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                               int H, bool active, int d0, const float (&cs)[8], const float (&sn)[8],
+                                               const Problem& P) {
+    using G = TokGeom<D>;
+    constexpr int kHalf = D / 2;
+    constexpr int kIn = 4;  // head rows in flight
+    for (int h0 = 0; h0 < H; h0 += kIn) {  // H is the same for every lane of the warp
+        float lo[kIn][8], hi[kIn][8];
+#pragma unroll
+        for (int j = 0; j < kIn; ++j) {
+            if (active && h0 + j < H) {
+                load_bf16x8(x + (size_t)(h0 + j) * D + d0, lo[j]);
+                load_bf16x8(x + (size_t)(h0 + j) * D + kHalf + d0, hi[j]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) lo[j][i] = hi[j][i] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kIn; ++j) {
+            float rs = 1.0f;
+            if (P.qk_norm) {
+                float ss = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss += lo[j][i] * lo[j][i] + hi[j][i] * hi[j][i];
+                ss = group_sum<G::GS>(ss);
+                rs = rsqrtf(ss * (1.0f / D) + P.eps);
+            }
+            if (!active || h0 + j >= H) continue;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a = lo[j][i] * rs, bb = hi[j][i] * rs;
+                lo[j][i] = a * cs[i] - bb * sn[i];
+                hi[j][i] = bb * cs[i] + a * sn[i];
+            }
+            store_bf16x8(y + (size_t)(h0 + j) * D + d0, lo[j]);
+            store_bf16x8(y + (size_t)(h0 + j) * D + kHalf + d0, hi[j]);
+        }
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ k,
                                                      __nv_bfloat16* __restrict__ qo, __nv_bfloat16* __restrict__ ko,
-                                                     Problem P, uint32_t rows_q, uint32_t rows_total) {
-    using G = RowGeom<D>;
-    constexpr int kHalf = D / 2;
+                                                     Problem P, const RopeFreq F, uint32_t tokens) {
+    using G = TokGeom<D>;
     const int g = threadIdx.x & (G::GS - 1);
-    const uint32_t row_raw = blockIdx.x * (uint32_t)G::ROWS + threadIdx.x / G::GS;
-    // no early return: every lane of the warp takes part in the group shuffles below
-    const bool valid = row_raw < rows_total;
-    const uint32_t row = valid ? row_raw : 0;
-    const bool is_q = row < rows_q;
-    const uint32_t r = is_q ? row : row - rows_q;
-    const uint32_t tok = fastdiv(r, is_q ? P.div_hq : P.div_hkv);  // b * T + t (queries: b * Tq + t)
-    const uint32_t b = fastdiv(tok, is_q ? P.div_tq : P.div_t);
-    const int t = (int)(tok - b * (uint32_t)(is_q ? P.Tq : P.T));
-    const __nv_bfloat16* x = (is_q ? q : k) + (size_t)r * D;
-    __nv_bfloat16* y = (is_q ? qo : ko) + (size_t)r * D;
+    const uint32_t tok_raw = blockIdx.x * (uint32_t)G::TOK + threadIdx.x / G::GS;  // b * Tq + t
+    // no early return: every lane of the warp takes part in the group shuffles
+    const bool valid = tok_raw < tokens;
+    const uint32_t tok = valid ? tok_raw : 0;
     const bool active = valid && g < G::LPR;
-    const int d0 = 8 * g;
-    float lo[8], hi[8];
-    float4 cs[4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) lo[i] = hi[i] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) cs[i] = make_float4(1.f, 0.f, 1.f, 0.f);
-    if (active) {
-        load_bf16x8(x + d0, lo);
-        load_bf16x8(x + kHalf + d0, hi);
-        if (P.rope) {  // issued together with the row loads: its latency overlaps theirs
-            // queries over a cache sit at qoff + t; segments only come without a cache
-            const int pos = P.seg_start ? t - P.seg_start[tok] : t + (is_q ? P.qoff : 0);
-            const float4* c = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cs[i] = c[i];
-        }
-    }
-    float rs = 1.0f;
-    if (P.qk_norm) {
-        float ss = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss += lo[i] * lo[i] + hi[i] * hi[i];
-        ss = group_sum<G::GS>(ss);
-        rs = rsqrtf(ss * (1.0f / D) + P.eps);
-    }
-    if (!active) return;
+    const int d0 = 8 * (active ? g : 0);
+    float cs[8], sn[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        lo[i] *= rs;
-        hi[i] *= rs;
+        cs[i] = 1.f;
+        sn[i] = 0.f;
     }
-    if (P.rope) {
+    if (P.rope && active) {
+        const uint32_t b = fastdiv(tok, P.div_tq);
+        const int t = (int)(tok - b * (uint32_t)P.Tq);
+        // queries over a cache sit at qoff + t; segments only come without a cache (Tq = T)
+        const int pos = P.seg_start ? t - P.seg_start[tok] : t + P.qoff;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float c = (i & 1) ? cs[i / 2].z : cs[i / 2].x;
-            const float sn = (i & 1) ? cs[i / 2].w : cs[i / 2].y;
-            const float a = lo[i], bb = hi[i];
-            lo[i] = a * c - bb * sn;
-            hi[i] = bb * c + a * sn;
+            const float2 a = rope_angle(pos, F.theta[d0 + i]);
+            cs[i] = a.x;
+            sn[i] = a.y;
         }
     }
-    store_bf16x8(y + d0, lo);
-    store_bf16x8(y + kHalf + d0, hi);
+    prologue_heads<D>(q + (size_t)tok * P.Hq * D, qo + (size_t)tok * P.Hq * D, P.Hq, active, d0, cs, sn, P);
+    // keys: same tokens (a key tensor is only passed without a cache, where Tq = T and qoff = 0)
+    if (k) prologue_heads<D>(k + (size_t)tok * P.Hkv * D, ko + (size_t)tok * P.Hkv * D, P.Hkv, active, d0, cs, sn, P);
 }
 
 // ------------------------------------------------------------------ backward preprocess
@@ -203,94 +211,128 @@ __global__ void __launch_bounds__(256) k_bwd_pre(const __nv_bfloat16* __restrict
 }
 
 // ------------------------------------------------------------------ gradient finalize
-// Rows [0, rows_q): dq = RMSNorm^T(RoPE^T(scale * dQ')) from the fp32 accumulator and raw q.
-// Rows [rows_q, rows_q + rows_k): the same for dk from raw dK' and raw k (only when QK-norm
-// or RoPE is on; otherwise the attention kernel already wrote dk).
+// dq = RMSNorm^T(RoPE^T(scale * dQ')) from the fp32 accumulator and raw q, for every query
+// head of a token; then the same for dk from raw dK' and raw k (only when QK-norm or RoPE is
+// on; otherwise the attention kernel already wrote dk).  A group of GS lanes owns one token;
+// a lane owns 4 rotation pairs (16-byte fp32 loads of each half) and forms their RoPE angles
+// once for the token.
+template <int D>
+struct FinGeom {
+    static constexpr int LPR = D / 8;
+    static constexpr int GS = (LPR <= 4) ? 4 : (LPR <= 8 ? 8 : 16);
+    static constexpr int TOK = 256 / GS;
+};
+
+template <int D>
+__device__ __forceinline__ void finalize_heads(const float* __restrict__ acc, const __nv_bfloat16* __restrict__ x,
+                                               __nv_bfloat16* __restrict__ out, int H, bool active, int d0,
+                                               const float (&cs)[4], const float (&sn)[4], const Problem& P) {
+    using G = FinGeom<D>;
+    constexpr int kHalf = D / 2;
+    constexpr int kIn = 4;
+    for (int h0 = 0; h0 < H; h0 += kIn) {
+        float u_lo[kIn][4], u_hi[kIn][4], x_lo[kIn][4], x_hi[kIn][4];
+#pragma unroll
+        for (int j = 0; j < kIn; ++j) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) u_lo[j][i] = u_hi[j][i] = x_lo[j][i] = x_hi[j][i] = 0.f;
+            if (active && h0 + j < H) {
+                const float* a = acc + (size_t)(h0 + j) * D;
+                const float4 l4 = *reinterpret_cast<const float4*>(a + d0);
+                const float4 h4 = *reinterpret_cast<const float4*>(a + kHalf + d0);
+                u_lo[j][0] = l4.x; u_lo[j][1] = l4.y; u_lo[j][2] = l4.z; u_lo[j][3] = l4.w;
+                u_hi[j][0] = h4.x; u_hi[j][1] = h4.y; u_hi[j][2] = h4.z; u_hi[j][3] = h4.w;
+                if (P.qk_norm) {
+                    load_bf16x4(x + (size_t)(h0 + j) * D + d0, x_lo[j]);
+                    load_bf16x4(x + (size_t)(h0 + j) * D + kHalf + d0, x_hi[j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kIn; ++j) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                u_lo[j][i] *= P.scale;
+                u_hi[j][i] *= P.scale;
+                rope_transpose(u_lo[j][i], u_hi[j][i], make_float2(cs[i], sn[i]));
+            }
+            if (P.qk_norm) {
+                float ss = 0.f, dot = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ss += x_lo[j][i] * x_lo[j][i] + x_hi[j][i] * x_hi[j][i];
+                    dot += u_lo[j][i] * x_lo[j][i] + u_hi[j][i] * x_hi[j][i];
+                }
+                ss = group_sum<G::GS>(ss);
+                dot = group_sum<G::GS>(dot);
+                const float rs = rsqrtf(ss * (1.0f / D) + P.eps);
+                const float k3 = rs * rs * rs * dot * (1.0f / D);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    u_lo[j][i] = rs * u_lo[j][i] - k3 * x_lo[j][i];
+                    u_hi[j][i] = rs * u_hi[j][i] - k3 * x_hi[j][i];
+                }
+            }
+            if (!active || h0 + j >= H) continue;
+            store_bf16x4(out + (size_t)(h0 + j) * D + d0, u_lo[j]);
+            store_bf16x4(out + (size_t)(h0 + j) * D + kHalf + d0, u_hi[j]);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__ dq_acc,
                                                        const float* __restrict__ dk_acc,
                                                        const __nv_bfloat16* __restrict__ q,
                                                        const __nv_bfloat16* __restrict__ k,
                                                        __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
-                                                       Problem P, uint32_t rows_q, uint32_t rows_total) {
-    constexpr int kHalf = D / 2;
-    const int lane16 = threadIdx.x & 15;
-    const uint32_t row_raw = blockIdx.x * 16u + (threadIdx.x >> 4);
-    const bool valid = row_raw < rows_total;  // no early return: the group shuffles need every lane
-    const uint32_t row0 = valid ? row_raw : 0;
-    const bool is_q = row0 < rows_q;
-    const size_t row = is_q ? row0 : row0 - rows_q;
-    const float* acc = is_q ? dq_acc : dk_acc;
-    const __nv_bfloat16* x = is_q ? q : k;
-    __nv_bfloat16* out = is_q ? dq : dk;
-    const bool active = valid && lane16 < D / 8;
-    const int d0 = 4 * lane16;
-    float u_lo[4] = {0.f, 0.f, 0.f, 0.f}, u_hi[4] = {0.f, 0.f, 0.f, 0.f};
-    float x_lo[4] = {0.f, 0.f, 0.f, 0.f}, x_hi[4] = {0.f, 0.f, 0.f, 0.f};
-    if (active) {
-        const float4 a = *reinterpret_cast<const float4*>(acc + row * D + d0);
-        const float4 c = *reinterpret_cast<const float4*>(acc + row * D + kHalf + d0);
-        u_lo[0] = a.x * P.scale; u_lo[1] = a.y * P.scale; u_lo[2] = a.z * P.scale; u_lo[3] = a.w * P.scale;
-        u_hi[0] = c.x * P.scale; u_hi[1] = c.y * P.scale; u_hi[2] = c.z * P.scale; u_hi[3] = c.w * P.scale;
-        if (P.qk_norm) {
-            load_bf16x4(x + row * D + d0, x_lo);
-            load_bf16x4(x + row * D + kHalf + d0, x_hi);
-        }
-        if (P.rope) {
-            const uint32_t tok = fastdiv((uint32_t)row, is_q ? P.div_hq : P.div_hkv);  // b * T + t
-            const int t = (int)(tok - fastdiv(tok, P.div_t) * (uint32_t)P.T);
-            const int pos = P.seg_start ? t - P.seg_start[tok] : t;
-            const float4* cs = reinterpret_cast<const float4*>(P.rope_cs + (size_t)pos * kHalf + d0);
-            const float4 c01 = cs[0], c23 = cs[1];
-            rope_transpose(u_lo[0], u_hi[0], make_float2(c01.x, c01.y));
-            rope_transpose(u_lo[1], u_hi[1], make_float2(c01.z, c01.w));
-            rope_transpose(u_lo[2], u_hi[2], make_float2(c23.x, c23.y));
-            rope_transpose(u_lo[3], u_hi[3], make_float2(c23.z, c23.w));
-        }
+                                                       Problem P, const RopeFreq F, uint32_t tokens) {
+    using G = FinGeom<D>;
+    const int g = threadIdx.x & (G::GS - 1);
+    const uint32_t tok_raw = blockIdx.x * (uint32_t)G::TOK + threadIdx.x / G::GS;  // b * T + t
+    const bool valid = tok_raw < tokens;  // no early return: the group shuffles need every lane
+    const uint32_t tok = valid ? tok_raw : 0;
+    const bool active = valid && g < G::LPR;
+    const int d0 = 4 * (active ? g : 0);
+    float cs[4], sn[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        cs[i] = 1.f;
+        sn[i] = 0.f;
     }
-    if (P.qk_norm) {
-        float ss = 0.f, dot = 0.f;
+    if (P.rope && active) {
+        const int t = (int)(tok - fastdiv(tok, P.div_t) * (uint32_t)P.T);
+        const int pos = P.seg_start ? t - P.seg_start[tok] : t;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            ss += x_lo[i] * x_lo[i] + x_hi[i] * x_hi[i];
-            dot += u_lo[i] * x_lo[i] + u_hi[i] * x_hi[i];
-        }
-        ss = group_sum<16>(ss);
-        dot = group_sum<16>(dot);
-        const float rs = rsqrtf(ss * (1.0f / D) + P.eps);
-        const float k3 = rs * rs * rs * dot * (1.0f / D);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            u_lo[i] = rs * u_lo[i] - k3 * x_lo[i];
-            u_hi[i] = rs * u_hi[i] - k3 * x_hi[i];
+            const float2 a = rope_angle(pos, F.theta[d0 + i]);
+            cs[i] = a.x;
+            sn[i] = a.y;
         }
     }
-    if (!active) return;
-    store_bf16x4(out + row * D + d0, u_lo);
-    store_bf16x4(out + row * D + kHalf + d0, u_hi);
+    const size_t oq = (size_t)tok * P.Hq * D;
+    finalize_heads<D>(dq_acc + oq, q + oq, dq + oq, P.Hq, active, d0, cs, sn, P);
+    if (dk_acc) {
+        const size_t ok = (size_t)tok * P.Hkv * D;
+        finalize_heads<D>(dk_acc + ok, k + ok, dk + ok, P.Hkv, active, d0, cs, sn, P);
+    }
 }
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end,
-                        float2* rope_cs, double rope_base, cudaStream_t st) {
-    const int half = P.D / 2;
-    const int seg_blocks = ids ? P.B : 0;
-    const long long rope_n = rope_cs ? (long long)P.T * half : 0;
-    const int rope_blocks = (int)((rope_n + 1023) / 1024);
-    if (seg_blocks + rope_blocks == 0) return cudaSuccess;
-    k_prep<<<seg_blocks + rope_blocks, 1024, 0, st>>>(P.B, P.T, ids, seg_start, seg_end, rope_cs, half,
-                                                       rope_base > 0 ? log(rope_base) : 0.0);
+cudaError_t launch_prep(const Problem& P, const int32_t* ids, int32_t* seg_start, int32_t* seg_end, cudaStream_t st) {
+    if (!ids || P.B == 0) return cudaSuccess;
+    k_prep<<<P.B, 1024, 0, st>>>(P.T, ids, seg_start, seg_end);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_prologue_d(const Problem& P, const void* q, const void* k, void* qo, void* ko,
                                      cudaStream_t st) {
-    const long long rows_q = (long long)P.B * P.Tq * P.Hq;
-    const long long rows = rows_q + (k ? (long long)P.B * P.T * P.Hkv : 0);  // k == null: queries only
-    const long long blocks = (rows + RowGeom<D>::ROWS - 1) / RowGeom<D>::ROWS;
-    k_qk_prologue<D><<<(unsigned)blocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, (uint32_t)rows_q, (uint32_t)rows);
+    const long long tokens = (long long)P.B * P.Tq;  // k == null: queries only (over a cache)
+    const long long blocks = (tokens + TokGeom<D>::TOK - 1) / TokGeom<D>::TOK;
+    const RopeFreq F = rope_freq(D, P.rope_log_base);
+    k_qk_prologue<D><<<(unsigned)blocks, 256, 0, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                      (__nv_bfloat16*)qo, (__nv_bfloat16*)ko, P, F, (uint32_t)tokens);
     return cudaGetLastError();
 }
 
@@ -306,12 +348,12 @@ static cudaError_t launch_bwd_pre_d(const Problem& P, const void* o, const void*
 template <int D>
 static cudaError_t launch_grad_finalize_d(const Problem& P, const float* dq_acc, const float* dk_acc, const void* q,
                                           const void* k, void* dq, void* dk, cudaStream_t st) {
-    const long long rows_q = (long long)P.B * P.T * P.Hq;
-    const long long rows_k = (P.rope || P.qk_norm) ? (long long)P.B * P.T * P.Hkv : 0;
-    const long long rows = rows_q + rows_k;
-    k_grad_finalize<D><<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(
-        dq_acc, dk_acc, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, P,
-        (uint32_t)rows_q, (uint32_t)rows);
+    const long long tokens = (long long)P.B * P.T;
+    const long long blocks = (tokens + FinGeom<D>::TOK - 1) / FinGeom<D>::TOK;
+    const RopeFreq F = rope_freq(D, P.rope_log_base);
+    k_grad_finalize<D><<<(unsigned)blocks, 256, 0, st>>>(
+        dq_acc, (P.rope || P.qk_norm) ? dk_acc : nullptr, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+        (__nv_bfloat16*)dq, (__nv_bfloat16*)dk, P, F, (uint32_t)tokens);
     return cudaGetLastError();
 }
 

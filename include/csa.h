@@ -27,8 +27,10 @@
  *    bf16 pointers are passed as void* and hold IEEE bfloat16 bit patterns.
  *  - Every tensor pointer is a DEVICE pointer, allocated and owned by the caller, aligned to
  *    16 bytes.  The workspace is caller-owned device memory of at least
- *    csa_workspace_size() bytes, aligned to 256 bytes.  The library allocates no device
- *    memory of its own in any call.
+ *    csa_workspace_size() bytes, aligned to 256 bytes.  No call allocates device memory.
+ *    The one piece of device memory the library owns is the fixed scratch array of
+ *    csa_attn_fwd_static_scratch (CSA_STATIC_SCRATCH_BYTES), a module-scope array that every
+ *    GPU holds once the library is loaded on it.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it and
  *    the call returns without synchronising.  The only call that synchronises is
  *    csa_device_status().
@@ -104,12 +106,12 @@ int csa_attn_bwd(const csa_params* p, const void* q, const void* k, const void* 
                  void* dv, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward that reuses what the forward left in the workspace: the normalised and rotated
- * q', k' (QK-norm / RoPE on), the segment bounds and the RoPE table, so no prologue runs
- * (a training step computes q', k' once, in its forward).  Same arguments and results as
- * csa_attn_bwd.  Contract: the workspace (sized with for_backward = 1) was passed to
- * csa_attn_fwd with the same *p, q, k and segment_ids, on the same stream, and nothing has
- * written to it since.  The library cannot check this; a broken contract gives wrong
- * gradients (every access stays inside the workspace), never a fault. */
+ * q', k' (QK-norm / RoPE on) and the segment bounds, so no prologue runs (a training step
+ * computes q', k' once, in its forward).  Same arguments and results as csa_attn_bwd.
+ * Contract: the workspace (sized with for_backward = 1) was passed to csa_attn_fwd with the
+ * same *p, q, k and segment_ids, on the same stream, and nothing has written to it since.
+ * The library cannot check this; a broken contract gives wrong gradients (every access
+ * stays inside the workspace), never a fault. */
 int csa_attn_bwd_after_fwd(const csa_params* p, const void* q, const void* k, const void* v,
                            const void* o, const void* dout, const float* lse,
                            const int32_t* segment_ids, void* dq, void* dk, void* dv,
@@ -175,16 +177,16 @@ const char* csa_status_string(int code);
  * such entry point; it has no counterpart there.
  *
  * Same arguments and results as csa_attn_fwd, minus the workspace.  Its scratch (status
- * word, segment bounds, RoPE table, normalised q/k copies) lives in one file-scope device
+ * word, segment bounds, normalised q/k copies) lives in one file-scope device
  * array of CSA_STATIC_SCRATCH_BYTES that every GPU loading the library holds until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
  * library routine.
  *  - A problem whose scratch would exceed CSA_STATIC_SCRATCH_BYTES (roughly
- *    B*T*(Hq+Hkv)*D*2 bytes with QK-norm or RoPE, plus 8*B*T with segment_ids and 4*T*D with
- *    RoPE) is rejected with CSA_ERR_WORKSPACE before anything is enqueued.
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *    with that device current and caches it; make that first call before any stream
- *    capture.
+ *    B*T*(Hq+Hkv)*D*2 bytes with QK-norm or RoPE, plus 8*B*T with segment_ids) is rejected
+ *    with CSA_ERR_WORKSPACE before anything is enqueued.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress) with the
+ *    caller's device current; the first call on a device also loads the library's module
+ *    there, so make that first call before any stream capture.
  *  - Every call shares the one array, which keeps the last call's contents.  The call
  *    clears the status word it needs at zero and rewrites everything else before reading
  *    it.  Calls that overlap on the GPU (different streams, or threads) race on the array

@@ -102,7 +102,7 @@ def test_status_strings(b):
         assert b.status_string(code)
     assert b.status_string(6) == "a bounded wait inside a kernel ran out"
     assert b.kernel_names() == ["k_prep", "k_qk_prologue", "k_attn_fwd", "k_bwd_pre", "k_attn_bwd",
-                                "k_grad_finalize", "k_decode_q", "k_decode_split"]
+                                "k_grad_finalize", "k_decode"]
 
 
 def test_decode_arguments_are_checked_on_the_host(b):
@@ -130,11 +130,11 @@ def test_prefill_arguments_are_checked_on_the_host(b):
     p = b.make_params(2, 512, 8, 4, 96, rope_base=10000.0, qk_norm=True)
     n = b.prefill_workspace_size(p, 128)
     assert n > 0
-    # RoPE table for the 512 cache positions plus q' of the 128-token chunk
-    assert n >= 512 * 48 * 8 + 2 * 128 * 8 * 96 * 2
+    # q' of the 128-token chunk (the RoPE angles are formed in the kernels, no table)
+    assert n >= 2 * 128 * 8 * 96 * 2
     assert b.prefill_workspace_size(p, 0) == 0
     assert b.prefill_workspace_size(p, 513) == 0
-    assert b.prefill_workspace_size(b.make_params(2, 512, 8, 4, 96), 128) < n  # no prologue, no table
+    assert b.prefill_workspace_size(b.make_params(2, 512, 8, 4, 96), 128) < n  # no prologue
     pre = b.lib.csa_attn_prefill
     ptr = [0x1000 * (i + 1) for i in range(6)]
     assert pre(ctypes.byref(p), 513, *ptr[:5], 0x10000, 1 << 30, None) == b.CSA_ERR_INVALID_ARG
