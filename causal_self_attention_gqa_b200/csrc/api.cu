@@ -162,7 +162,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // [B, T, H, D] bf16 tensor, boxes of (swizzle-atom width) x 1 head x 128 rows x 1 batch.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+// promote: L2 fills of 256 bytes around each box row -- right when the other heads of the same
+// tokens are read at about the same time (the attention kernels), wasted bytes when they are
+// not (the decode kernel streams one head of a token long before or after its neighbours).
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D, bool promote = true) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const int sw = (D % 64 == 0) ? 128 : 64;
@@ -173,7 +176,8 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
                           sw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          promote ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -514,7 +518,8 @@ int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_ca
     int* done = reinterpret_cast<int*>(w + kAlign);
     float* part = reinterpret_cast<float*>(w + kAlign + up(d.done_bytes));
     CUtensorMap tk, tv;
-    if (!make_map(&tk, k_cache, p->B, p->T, p->Hkv, p->D) || !make_map(&tv, v_cache, p->B, p->T, p->Hkv, p->D))
+    if (!make_map(&tk, k_cache, p->B, p->T, p->Hkv, p->D, false) ||
+        !make_map(&tv, v_cache, p->B, p->T, p->Hkv, p->D, false))
         return CSA_ERR_CUDA;
     // status word and range counters start at zero
     if (cudaMemsetAsync(w, 0, kAlign + d.done_bytes, st) != cudaSuccess) {

@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(512, 1)
                         tma_store_4d(&tm_dk, smem + C::OFF_K + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
                 }
                 bulk_commit_group();
-                bulk_wait_group0();
+                bulk_wait_group_read0();  // the global writes complete with the grid
             }
         }
     } else if (warp >= 12) {
@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
         }
-        if (r == 0) bulk_wait_group0();
+        if (r == 0) bulk_wait_group_read0();  // the global writes complete with the grid
     }
 
     tc_fence_before();

@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive(&o_turn[i]);  // staging read: the other warpgroup's turn
             }
         }
-        if (r == 0) bulk_wait_group0();
+        if (r == 0) bulk_wait_group_read0();  // the global writes complete with the grid
     }
 
     tc_fence_before();

@@ -144,7 +144,7 @@ __device__ __forceinline__ void prologue_heads(const __nv_bfloat16* __restrict__
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) k_qk_prologue(const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(256, 3) k_qk_prologue(const __nv_bfloat16* __restrict__ q,
                                                      const __nv_bfloat16* __restrict__ k,
                                                      __nv_bfloat16* __restrict__ qo, __nv_bfloat16* __restrict__ ko,
                                                      Problem P, const RopeFreq F, uint32_t tokens) {
@@ -223,13 +223,14 @@ struct FinGeom {
     static constexpr int TOK = 256 / GS;
 };
 
+// Two head rows in flight per lane (64 registers, four 256-thread blocks per SM).
 template <int D>
 __device__ __forceinline__ void finalize_heads(const float* __restrict__ acc, const __nv_bfloat16* __restrict__ x,
                                                __nv_bfloat16* __restrict__ out, int H, bool active, int d0,
                                                const float (&cs)[4], const float (&sn)[4], const Problem& P) {
     using G = FinGeom<D>;
     constexpr int kHalf = D / 2;
-    constexpr int kIn = 4;
+    constexpr int kIn = 2;
     for (int h0 = 0; h0 < H; h0 += kIn) {
         float u_lo[kIn][4], u_hi[kIn][4], x_lo[kIn][4], x_hi[kIn][4];
 #pragma unroll
@@ -281,7 +282,7 @@ __device__ __forceinline__ void finalize_heads(const float* __restrict__ acc, co
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) k_grad_finalize(const float* __restrict__ dq_acc,
+__global__ void __launch_bounds__(256, 4) k_grad_finalize(const float* __restrict__ dq_acc,
                                                        const float* __restrict__ dk_acc,
                                                        const __nv_bfloat16* __restrict__ q,
                                                        const __nv_bfloat16* __restrict__ k,
