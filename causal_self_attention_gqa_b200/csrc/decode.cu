@@ -19,8 +19,9 @@
 //     swizzled 128-row boxes as the attention kernels) into a ring of K/V stages, so several
 //     chunks are in flight per CTA at any time;
 //   * four compute warps take 32 keys of each chunk: lane = key for the scores (rows of the
-//     swizzled tile read without bank conflicts), lane = 4 dimensions for P V, online
-//     softmax in log2 units;
+//     swizzled tile read without bank conflicts, the q' rows 16 bytes at a time, packed
+//     f32x2 FMAs), lane = 4 dimensions for P V (the probabilities of four keys at a time
+//     read back from shared memory), online softmax in log2 units;
 //   * the CTA's partial (m, l, o) goes to the workspace, and the last CTA of each
 //     (b, kv head) to count itself done merges every range: o = sum 2^(m_s - m) o_s / l.
 //     It also resets that counter, so the next call needs no clearing pass.
@@ -51,7 +52,8 @@ struct DecCfg {
     static constexpr int OFF_Q = OFF_KV + STAGES * 2 * TILE;           // q' [RMAX][D] fp32
     static constexpr int OFF_WO = OFF_Q + RMAX * D * 4;                // [4][RMAX][D] fp32
     static constexpr int OFF_WML = OFF_WO + kDecWarps * RMAX * D * 4;  // m, l [4][RMAX] each
-    static constexpr int OFF_BAR = OFF_WML + 2 * kDecWarps * RMAX * 4;
+    static constexpr int OFF_PS = OFF_WML + 2 * kDecWarps * RMAX * 4;  // p of a warp's keys [4][RMAX][32]
+    static constexpr int OFF_BAR = OFF_PS + kDecWarps * RMAX * 32 * 4;
     static constexpr int NBAR = 2 * STAGES;                            // full[S], empty[S]
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;                // abort flag, last flag
     static constexpr int SMEM = OFF_MISC + 16;
@@ -71,22 +73,41 @@ struct DecArgs {
 
 // o and LSE of one (b, kv head) from the partials of all its key ranges:
 // m = max_s m_s, l = sum_s 2^(m_s - m) l_s, o = sum_s 2^(m_s - m) o_s / l.  The partials come
-// from other CTAs: read through L2 (ld.global.cg), never from this SM's L1.
+// from other CTAs: read through L2 (ld.global.cg), never from this SM's L1, eight ranges'
+// values at a time with every load issued before the first use (a range's loads do not wait
+// for the previous range's).
 template <int D>
 __device__ void merge_partials(const DecArgs& A, int b, int kvh) {
     const Problem& P = A.P;
     const float* src = A.part + (((size_t)b * P.Hkv + kvh) * A.splits) * A.R * (D + 2);
+    constexpr int kBatch = 8;
     for (int e = threadIdx.x; e < A.R * D; e += blockDim.x) {
         const int r = e / D, d = e % D;
-        float mm = -INFINITY;
-        for (int s = 0; s < A.splits; ++s) mm = fmaxf(mm, __ldcg(src + ((size_t)s * A.R + r) * (D + 2) + D));
-        float acc = 0.f, ll = 0.f;
-        for (int s = 0; s < A.splits; ++s) {
-            const float* ps = src + ((size_t)s * A.R + r) * (D + 2);
-            const float ms = __ldcg(ps + D);
-            const float f = (ms == -INFINITY) ? 0.f : ex2(ms - mm);
-            acc += f * __ldcg(ps + d);
-            ll += f * __ldcg(ps + D + 1);
+        float mm = -INFINITY, acc = 0.f, ll = 0.f;
+        for (int s0 = 0; s0 < A.splits; s0 += kBatch) {
+            float ms[kBatch], os[kBatch], ls[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const float* ps = src + ((size_t)(s0 + u) * A.R + r) * (D + 2);
+                const bool in = s0 + u < A.splits;
+                ms[u] = in ? __ldcg(ps + D) : -INFINITY;
+                os[u] = in ? __ldcg(ps + d) : 0.f;
+                ls[u] = in ? __ldcg(ps + D + 1) : 0.f;
+            }
+            float bm = mm;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) bm = fmaxf(bm, ms[u]);
+            // rescale what is summed so far to the new reference max, then add this batch
+            const float f0 = (mm == -INFINITY) ? 0.f : ex2(mm - bm);
+            acc *= f0;
+            ll *= f0;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const float f = (ms[u] == -INFINITY) ? 0.f : ex2(ms[u] - bm);
+                acc += f * os[u];
+                ll += f * ls[u];
+            }
+            mm = bm;
         }
         const int i = r % A.Tq, h = kvh * P.G + r / A.Tq;
         A.o[((size_t)(b * A.Tq + i) * P.Hq + h) * D + d] = __float2bfloat16_rn(ll > 0.f ? acc / ll : 0.f);
@@ -131,6 +152,7 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
     float(*wo)[RMAX][D] = reinterpret_cast<float(*)[RMAX][D]>(smem + C::OFF_WO);
     float(*wm)[RMAX] = reinterpret_cast<float(*)[RMAX]>(smem + C::OFF_WML);
     float(*wl)[RMAX] = reinterpret_cast<float(*)[RMAX]>(smem + C::OFF_WML + kDecWarps * RMAX * 4);
+    float(*psh)[RMAX][32] = reinterpret_cast<float(*)[RMAX][32]>(smem + C::OFF_PS);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + C::STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
@@ -215,13 +237,13 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
         named_bar_sync(1, 32 * kDecWarps);
 
         const float kLog2e = 1.4426950408889634f;
-        float m[RMAX], l[RMAX], acc[RMAX][4];
+        float m[RMAX], l[RMAX];
+        float2 acc[RMAX][2];  // dimensions 4 lane + {0, 1}, 4 lane + {2, 3}
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) {
             m[r] = -INFINITY;
             l[r] = 0.f;
-#pragma unroll
-            for (int t = 0; t < 4; ++t) acc[r][t] = 0.f;
+            acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
         }
         const bool pv_lane = 4 * lane < D;  // lane owns dimensions [4 lane, 4 lane + 4) in P V
         const int row = 32 * warp + lane;    // this lane's key row in every chunk (scores)
@@ -233,25 +255,32 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
             const int k0 = k_begin + c * kDecChunk + 32 * warp;  // this warp's first key
             const int key = k0 + lane;
             const bool kin = key < k_end;
-            // scores of this lane's key against every row (q' rows broadcast from shared memory)
-            float sc[RMAX];
+            // scores of this lane's key against every row (q' rows broadcast from shared memory,
+            // 16 bytes at a time; products of element pairs with packed f32x2 FMAs)
+            float2 sc2[RMAX];
 #pragma unroll
-            for (int r = 0; r < RMAX; ++r) sc[r] = 0.f;
+            for (int r = 0; r < RMAX; ++r) sc2[r] = make_float2(0.f, 0.f);
 #pragma unroll 4
             for (int d8 = 0; d8 < D; d8 += 8) {
                 const uint4 u = *reinterpret_cast<const uint4*>(kt + swz_off<C::SW>(row, d8));
                 const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-                float kf[8];
+                float2 kf[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    kf[2 * e] = __uint_as_float(wv[e] << 16);
-                    kf[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
+                for (int e = 0; e < 4; ++e)
+                    kf[e] = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xffff0000u));
+#pragma unroll
+                for (int r = 0; r < RMAX; ++r) {
+                    const float4 qa = *reinterpret_cast<const float4*>(&qsh[r][d8]);
+                    const float4 qb = *reinterpret_cast<const float4*>(&qsh[r][d8 + 4]);
+                    sc2[r] = ffma2(make_float2(qa.x, qa.y), kf[0], sc2[r]);
+                    sc2[r] = ffma2(make_float2(qa.z, qa.w), kf[1], sc2[r]);
+                    sc2[r] = ffma2(make_float2(qb.x, qb.y), kf[2], sc2[r]);
+                    sc2[r] = ffma2(make_float2(qb.z, qb.w), kf[3], sc2[r]);
                 }
-#pragma unroll
-                for (int r = 0; r < RMAX; ++r)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) sc[r] = fmaf(qsh[r][d8 + e], kf[e], sc[r]);
             }
+            float sc[RMAX];
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) sc[r] = sc2[r].x + sc2[r].y;
             // logits in log2 units, masked to -inf
             float x[RMAX];
 #pragma unroll
@@ -276,26 +305,39 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
                 for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
                 if (mn != -INFINITY) {
                     l[r] = l[r] * alpha + ps;
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) acc[r][t] *= alpha;
+                    const float2 a2 = make_float2(alpha, alpha);
+                    acc[r][0] = fmul2(acc[r][0], a2);
+                    acc[r][1] = fmul2(acc[r][1], a2);
                     m[r] = mn;
                 }
+                psh[warp][r][lane] = p[r];
             }
-            // P V: key kk's probabilities broadcast from lane kk; lane owns 4 consecutive dims
-            const int nk = max(0, min(32, k_end - k0));
-#pragma unroll 4
-            for (int kk = 0; kk < nk; ++kk) {
-                uint2 vu = make_uint2(0u, 0u);
-                if (pv_lane) vu = *reinterpret_cast<const uint2*>(vt + swz_off<C::SW>(32 * warp + kk, 4 * lane));
-                const float vf[4] = {__uint_as_float(vu.x << 16), __uint_as_float(vu.x & 0xffff0000u),
-                                     __uint_as_float(vu.y << 16), __uint_as_float(vu.y & 0xffff0000u)};
+            __syncwarp();
+            // P V: lane owns 4 consecutive dims; the probabilities of four keys at a time are
+            // read back from shared memory (keys past the range have p = 0 and finite rows)
+            const int nk4 = (max(0, min(32, k_end - k0)) + 3) & ~3;
+            if (pv_lane) {
+#pragma unroll 2
+                for (int k4 = 0; k4 < nk4; k4 += 4) {
+                    float4 p4[RMAX];
 #pragma unroll
-                for (int r = 0; r < RMAX; ++r) {
-                    const float pk = __shfl_sync(0xffffffffu, p[r], kk);
+                    for (int r = 0; r < RMAX; ++r) p4[r] = *reinterpret_cast<const float4*>(&psh[warp][r][k4]);
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) acc[r][t] = fmaf(pk, vf[t], acc[r][t]);
+                    for (int u = 0; u < 4; ++u) {
+                        const uint2 vu = *reinterpret_cast<const uint2*>(vt + swz_off<C::SW>(32 * warp + k4 + u, 4 * lane));
+                        const float2 v01 = make_float2(__uint_as_float(vu.x << 16), __uint_as_float(vu.x & 0xffff0000u));
+                        const float2 v23 = make_float2(__uint_as_float(vu.y << 16), __uint_as_float(vu.y & 0xffff0000u));
+#pragma unroll
+                        for (int r = 0; r < RMAX; ++r) {
+                            const float pk = (u == 0) ? p4[r].x : (u == 1) ? p4[r].y : (u == 2) ? p4[r].z : p4[r].w;
+                            const float2 pk2 = make_float2(pk, pk);
+                            acc[r][0] = ffma2(pk2, v01, acc[r][0]);
+                            acc[r][1] = ffma2(pk2, v23, acc[r][1]);
+                        }
+                    }
                 }
             }
+            __syncwarp();            // psh is rewritten by the next chunk
             warp_arrive(&empty[s]);  // this warp is done with the stage
         }
         // this warp's partial to shared memory
@@ -306,8 +348,8 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
                 wl[warp][r] = l[r];
             }
             if (pv_lane)
-#pragma unroll
-                for (int t = 0; t < 4; ++t) wo[warp][r][4 * lane + t] = acc[r][t];
+                *reinterpret_cast<float4*>(&wo[warp][r][4 * lane]) =
+                    make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
         }
     }
     __syncthreads();

@@ -62,6 +62,9 @@ CASES = [
     (2, 513, 3, 4, 2, 32, dict(causal=False, window=100)),
     (1, 640, 8, 2, 1, 128, dict(softcap=5.0, scale=0.05)),
     (2, 100000, 1, 8, 4, 96, dict(rope_base=10000.0, qk_norm=True)),  # RoPE at positions near 1e5
+    # several blocks of adjacent kv heads per token (4 + 4, and 2 + 2 + 2)
+    (2, 700, 1, 16, 8, 64, dict(rope_base=10000.0, qk_norm=True)),
+    (1, 301, 2, 12, 6, 32, dict(window=150)),
 ]
 
 
