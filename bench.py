@@ -345,7 +345,8 @@ def measure_decode(steps: int, warmup: int, batch: int = 0) -> dict:
         "tokens_per_s": w.B * w.Tq / (ms * 1e-3),
         "kernels": {n: {"ms_avg": t / c if c else 0.0, "launches": c} for n, (t, c) in kt.items() if c},
         "roofline": {"bound": "hbm", "achieved": split_gbs, "peak": hbm, "unit": "GB/s", "frac": split_gbs / hbm,
-                     "traffic": None, "kernel": "k_decode", "peak_source": f"{src}, hbm_gbs"},
+                     "traffic": recorded_traffic("k_decode", w.name) if batch <= 0 else None,
+                     "kernel": "k_decode", "peak_source": f"{src}, hbm_gbs"},
         "gpu_launches": sum(c for _, c in kt.values()),
     }
     return line
