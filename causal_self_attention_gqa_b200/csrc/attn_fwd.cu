@@ -43,6 +43,8 @@
 
 namespace csa {
 
+constexpr int kItemWords = 10;  // item ring slot: index, then the fields of FwdItem
+
 template <int D>
 struct FwdCfg {
     static constexpr int SW = (D % 64 == 0) ? 128 : 64;  // swizzle span (bytes) of a tile row
@@ -60,8 +62,9 @@ struct FwdCfg {
     // o_full[2], o_empty[2], item_full[2], item_empty[2]
     // o_turn[2] (staging hand-off between the two warpgroups), ep_sync[2]
     static constexpr int NBAR = 2 + 3 * STAGES + 16;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, item ring [2]
-    static constexpr int SMEM = OFF_MISC + 32;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+    static constexpr int OFF_RING = OFF_MISC + 16;       // item ring [2][kItemWords]
+    static constexpr int SMEM = OFF_RING + 2 * kItemWords * 4;
     static constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
     static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, false, true);
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -103,12 +106,15 @@ __device__ __forceinline__ float capped_log2(float raw, const Problem& P) {
     return P.cap_log2 * tanh_approx(raw * P.cap_in);
 }
 
-// One work item, decoded identically by every role from its index.
+// One work item.  The producer decodes it once and publishes the fields in the item ring
+// (the code runs once per item, so in the consumers it would run cold, out of the
+// instruction cache).
 struct FwdItem {
     int b, kvh, hh[2], mm[2];
     bool two;
     int kt_begin, nkt;
 };
+
 
 __device__ __forceinline__ FwdItem decode_item(const FwdArgs& A, int idx) {
     const Problem& P = A.P;
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* ep_sync = s_full + 14;               // [2] warpgroup i has staged its O tile
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
+    volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_RING);  // [2][kItemWords]
 
     // the swizzled tiles need a 1024-byte aligned base; the condition is uniform over the CTA
     if ((smem_u32(smem) & 1023u) != 0) {
@@ -211,10 +217,20 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // next item index from the ring (slot n & 1); -1 ends the loop
-    auto take_item = [&](int n, int& idx) -> bool {
+    // next item from the ring (slot n & 1); index -1 ends the loop
+    auto take_item = [&](int n, int& idx, FwdItem& w) -> bool {
         if (!mbar_wait(&item_full[n & 1], (n >> 1) & 1, abort_flag, P.status)) return false;
-        idx = item_ring[n & 1];
+        const volatile int* r = item_ring + (n & 1) * kItemWords;
+        idx = r[0];
+        w.b = r[1];
+        w.kvh = r[2];
+        w.hh[0] = r[3];
+        w.hh[1] = r[4];
+        w.mm[0] = r[5];
+        w.mm[1] = r[6];
+        w.two = r[7] != 0;
+        w.kt_begin = r[8];
+        w.nkt = r[9];
         return true;
     };
 
@@ -229,10 +245,25 @@ __global__ void __launch_bounds__(384, 1)
                 const int idx = atomicAdd(A.counter, 1);
                 const int slot = n & 1;
                 if (n >= 2 && !mbar_wait(&item_empty[slot], ((n >> 1) - 1) & 1, abort_flag, P.status)) break;
-                item_ring[slot] = (idx < A.items) ? idx : -1;
+                volatile int* r = item_ring + slot * kItemWords;
+                FwdItem w{};
+                if (idx < A.items) {
+                    w = decode_item(A, idx);
+                    r[0] = idx;
+                    r[1] = w.b;
+                    r[2] = w.kvh;
+                    r[3] = w.hh[0];
+                    r[4] = w.hh[1];
+                    r[5] = w.mm[0];
+                    r[6] = w.mm[1];
+                    r[7] = w.two ? 1 : 0;
+                    r[8] = w.kt_begin;
+                    r[9] = w.nkt;
+                } else {
+                    r[0] = -1;
+                }
                 mbar_arrive(&item_full[slot]);
                 if (idx >= A.items) break;
-                const FwdItem w = decode_item(A, idx);
                 // Q tiles of this item once the previous item's last S MMA has read the old ones
                 if (n >= 1 && !mbar_wait(q_empty, (n - 1) & 1, abort_flag, P.status)) break;
                 mbar_arrive_expect_tx(q_full, (w.two ? 2 : 1) * C::TILE);
@@ -288,10 +319,10 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             for (int n = 0; ok; ++n) {
                 int idx;
-                if (!(ok = take_item(n, idx))) break;
+                FwdItem w;
+                if (!(ok = take_item(n, idx, w))) break;
                 mbar_arrive(&item_empty[n & 1]);
                 if (idx < 0) break;
-                const FwdItem w = decode_item(A, idx);
                 if (!(ok = mbar_wait(q_full, n & 1, abort_flag, P.status) &&
                            mbar_wait(&k_full[g % C::STAGES], (g / C::STAGES) & 1, abort_flag, P.status)))
                     break;
@@ -342,10 +373,10 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int n = 0; ok; ++n) {
             int idx = -1;
-            ok = __all_sync(0xffffffffu, take_item(n, idx));
+            FwdItem w;
+            ok = __all_sync(0xffffffffu, take_item(n, idx, w));
             warp_arrive(&item_empty[n & 1]);
             if (!ok || idx < 0) break;
-            const FwdItem w = decode_item(A, idx);
             if (i == 1 && !w.two) {
                 // no second tile in this item: pass the staging turn straight back
                 if (r == 0) {
