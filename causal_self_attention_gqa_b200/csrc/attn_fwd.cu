@@ -267,10 +267,13 @@ __global__ void __launch_bounds__(384, 1)
                 // Q tiles of this item once the previous item's last S MMA has read the old ones
                 if (n >= 1 && !mbar_wait(q_empty, (n - 1) & 1, abort_flag, P.status)) break;
                 mbar_arrive_expect_tx(q_full, (w.two ? 2 : 1) * C::TILE);
-                for (int i = 0; i < (w.two ? 2 : 1); ++i)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (i == 1 && !w.two) break;
                     for (int a = 0; a < C::NA; ++a)
                         tma_load_4d(&tm_q, q_full, smem + C::OFF_Q + i * C::TILE + a * kBM * C::SW, a * C::AE,
                                     w.hh[i], w.mm[i] * kBM, w.b);
+                }
                 bool ok = true;
                 for (int jj = 0; jj < w.nkt; ++jj, ++g) {
                     const int s = g % C::STAGES;
@@ -334,7 +337,10 @@ __global__ void __launch_bounds__(384, 1)
                     const int s = g % C::STAGES, ph = (g / C::STAGES) & 1;
                     const bool next = jj + 1 < w.nkt;
                     const int s2 = (g + 1) % C::STAGES, ph2 = ((g + 1) / C::STAGES) & 1;
-                    for (int i = 0; i < (w.two ? 2 : 1); ++i) {
+                    // i is a compile-time index (unrolled), so ps[] and no[] stay in registers
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (i == 1 && !w.two) break;
                         ok = mbar_wait(&v_full[s], ph, abort_flag, P.status) &&
                              mbar_wait(&p_full[i], ps[i] & 1, abort_flag, P.status);
                         // the first PV of an item overwrites O_i: the previous epilogue must have read it
@@ -347,16 +353,16 @@ __global__ void __launch_bounds__(384, 1)
                             if (i == 0 && !(ok = mbar_wait(&k_full[s2], ph2, abort_flag, P.status))) break;
                             tc_fence_after();
                             issue_s(i, s2);
+                        } else {
+                            // tile i's output is complete with this PV: its epilogue need not
+                            // wait for the other tile's last softmax
+                            umma_commit(&o_full[i]);
+                            ++no[i];
                         }
                     }
                     if (!ok) break;
                     if (jj + 2 == w.nkt) umma_commit(q_empty);  // the item's last S MMAs are issued
                     umma_commit(&kv_empty[s]);
-                }
-                if (!ok) break;
-                for (int i = 0; i < (w.two ? 2 : 1); ++i) {
-                    umma_commit(&o_full[i]);
-                    ++no[i];
                 }
             }
         }
@@ -387,8 +393,10 @@ __global__ void __launch_bounds__(384, 1)
                 ++nt;
                 continue;
             }
-            const int h = w.hh[i];
-            const int q = w.mm[i] * kBM + r;
+            // selects, not w.hh[i]: a runtime index would put the item in local memory
+            const int h = i ? w.hh[1] : w.hh[0];
+            const int m0 = i ? w.mm[1] : w.mm[0];
+            const int q = m0 * kBM + r;
             int lo, hi;
             row_bounds(P, w.b, q, lo, hi);
             float m_used = -INFINITY, l = 0.f;
@@ -541,7 +549,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             if (r == 0) {
                 for (int a = 0; a < C::NA; ++a)
-                    tma_store_4d(&tm_o, smem + C::OFF_O + a * kBM * C::SW, a * C::AE, h, w.mm[i] * kBM, w.b);
+                    tma_store_4d(&tm_o, smem + C::OFF_O + a * kBM * C::SW, a * C::AE, h, m0 * kBM, w.b);
                 bulk_commit_group();
                 bulk_wait_group_read0();
                 mbar_arrive(&o_turn[i]);  // staging read: the other warpgroup's turn
