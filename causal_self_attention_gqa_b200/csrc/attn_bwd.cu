@@ -205,12 +205,13 @@ __global__ void __launch_bounds__(512, 1)
                 tma_load_4d(&tm_k, kv_full, smem + C::OFF_K + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
                 tma_load_4d(&tm_v, kv_full, smem + C::OFF_V + a * kBM * C::SW, a * C::AE, kvh, n * kBN, b);
             }
-            for (int it = 0; it < nit; ++it) {
+            // iteration it is query head h of the group and query tile m (h = it / nm, m = m_lo +
+            // it % nm, kept as counters: no division per iteration)
+            int h = kvh * P.G, m = m_lo;
+            for (int it = 0; it < nit; ++it, (++m > m_lo + nm - 1) ? (m = m_lo, ++h) : 0) {
                 const int s = it % NS;
                 const uint32_t ph = ((it / NS) - 1) & 1;
                 if (it >= NS && !mbar_wait(&q_empty[s], ph, abort_flag, P.status)) break;
-                const int h = kvh * P.G + it / nm;
-                const int m = m_lo + it % nm;
                 mbar_arrive_expect_tx(&q_full[s], C::TILE);
                 for (int a = 0; a < C::NA; ++a)
                     tma_load_4d(&tm_q, &q_full[s], smem + C::OFF_Q + s * C::TILE + a * kBM * C::SW, a * C::AE, h,
@@ -326,22 +327,30 @@ __global__ void __launch_bounds__(512, 1)
         bool ok = nit > 0;
         // this thread's LSE (log2 units) and delta for query row kr of iteration `it`, loaded
         // from global one iteration ahead so the load latency hides behind the compute
-        auto fetch = [&](int it, float& l2, float& d) {
-            const int h = kvh * P.G + it / nm;
-            const int q = (m_lo + it % nm) * kBM + kr;
-            const size_t o = ((size_t)b * P.Hq + h) * P.T + (q < P.T ? q : 0);
+        // (head, query tile) of an iteration advance as counters: no division per iteration
+        const int m_last = m_lo + nm - 1;
+        int fh = kvh * P.G, fm = m_lo;  // the iteration fetched next
+        auto fetch = [&](float& l2, float& d) {
+            const int q = fm * kBM + kr;
+            const size_t o = ((size_t)b * P.Hq + fh) * P.T + (q < P.T ? q : 0);
             l2 = (q < P.T) ? A.lse[o] * kLog2e : INFINITY;
             d = (q < P.T) ? A.delta[o] : 0.f;
+            if (++fm > m_last) {
+                fm = m_lo;
+                ++fh;
+            }
         };
         float nl2 = INFINITY, nd = 0.f;
-        if (nit > 0) fetch(0, nl2, nd);
+        if (nit > 0) fetch(nl2, nd);
+        int cur_m = m_lo;
         for (int it = 0; ok && it < nit; ++it) {
-            const int m = m_lo + it % nm;
+            const int m = cur_m;
+            cur_m = (cur_m == m_last) ? m_lo : cur_m + 1;
             const int q0 = m * kBM;
             const int buf = it & 1;
             if (half == 0) lse_s[buf * 128 + kr] = nl2;
             else delta_s[buf * 128 + kr] = nd;
-            if (it + 1 < nit) fetch(it + 1, nl2, nd);
+            if (it + 1 < nit) fetch(nl2, nd);
             warp_arrive(wg_sync);
             ok = mbar_wait(wg_sync, it & 1, abort_flag, P.status);
             ok = ok && mbar_wait(s_full, it & 1, abort_flag, P.status);
@@ -550,10 +559,11 @@ __global__ void __launch_bounds__(512, 1)
             dph ^= 1u;
             return w;
         };
-        for (int it = 0; ok && it < nit; ++it) {
+        // (head, query tile) of an iteration as counters: no division per iteration
+        int h = kvh * P.G, m = m_lo;
+        for (int it = 0; ok && it < nit; ++it, (++m > m_lo + nm - 1) ? (m = m_lo, ++h) : 0) {
             const int s = it % NS;
-            const int h = kvh * P.G + it / nm;
-            const int q0 = (m_lo + it % nm) * kBM;
+            const int q0 = m * kBM;
             ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag, P.status));
             if (!ok) break;
             tc_fence_after();
