@@ -429,12 +429,15 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
                 const bool full = (k0 >= lo) && (k0 + kBN - 1 <= hi);
-                if (!full) {
+                const bool masked = !__all_sync(0xffffffffu, full);
+                if (masked) {
+                    // visible columns [a, a + span] of this tile, one unsigned compare per key (an
+                    // empty row, lo > hi, masks every key)
+                    const int a = (lo <= hi) ? lo - k0 : (1 << 20);
+                    const unsigned span = (lo <= hi) ? (unsigned)(hi - lo) : 0u;
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const int key = k0 + c;
-                        if (key < lo || key > hi) raw[c] = 0xff800000u;  // -inf
-                    }
+                    for (int c = 0; c < 128; ++c)
+                        if ((unsigned)(c - a) > span) raw[c] = 0xff800000u;  // -inf
                 }
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -457,12 +460,14 @@ __global__ void __launch_bounds__(384, 1)
                 const float nbase = (m_used == -INFINITY) ? 0.f : -m_used;
                 const float2 xm2 = make_float2(xmul, xmul), nb2 = make_float2(nbase, nbase);
                 float2 rsa = make_float2(0.f, 0.f), rsb = make_float2(0.f, 0.f);
-                // p = 2^(x - m): MUFU for most pairs; in tiles with no masked key (warp-uniform)
-                // one pair in four goes to the FMA pipe so both units share the work (one in
-                // two when tanh takes a MUFU slot too; none when the series tanh already loads
-                // the FMA pipe)
-                auto exp_pass = [&](auto emu_tag) {
-                    constexpr bool kEmu = decltype(emu_tag)::value;
+                // p = 2^(x - m): MUFU for most pairs; one pair in four goes to the FMA pipe so
+                // both units share the work (one in two when tanh takes a MUFU slot too; none
+                // when the series tanh already loads the FMA pipe).  In a tile with masked keys
+                // (kFull false) the FMA-pipe result of a masked key (x = -inf, clamped to -126)
+                // is set back to exactly 0.
+                auto exp_pass = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
+                    constexpr bool kEmu = true;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t pk[16];
@@ -472,10 +477,15 @@ __global__ void __launch_bounds__(384, 1)
                                                                 __uint_as_float(raw[32 * c + 2 * e + 1])),
                                                     xm2, nb2);
                             float2 pv;
-                            if (kEmu && (CM == 1 ? (e & 1) == 1 : (CM == 0 && (e & 3) == 3)))
+                            if (kEmu && (CM == 1 ? (e & 1) == 1 : (CM == 0 && (e & 3) == 3))) {
                                 pv = exp2_fma2(make_float2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f)));
-                            else
+                                if constexpr (!kFull) {
+                                    if (xv.x == -INFINITY) pv.x = 0.f;
+                                    if (xv.y == -INFINITY) pv.y = 0.f;
+                                }
+                            } else {
                                 pv = make_float2(ex2(xv.x), ex2(xv.y));
+                            }
                             if (e & 1) rsb = fadd2(rsb, pv);
                             else rsa = fadd2(rsa, pv);
                             pk[e] = pack_bf16x2(pv.x, pv.y);
@@ -483,7 +493,7 @@ __global__ void __launch_bounds__(384, 1)
                         tmem_st16(tS + 16 * c, pk);
                     }
                 };
-                if (__all_sync(0xffffffffu, full)) exp_pass(std::true_type{});
+                if (!masked) exp_pass(std::true_type{});
                 else exp_pass(std::false_type{});
                 const float rs = (rsa.x + rsa.y) + (rsb.x + rsb.y);
                 l = l * alpha + rs;
