@@ -357,7 +357,11 @@ __global__ void __launch_bounds__(512, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            const bool full = (q0 >= lo) && (q0 + kBM - 1 <= hi);
+            // masked tile (warp-uniform): query column k is visible when k - (lo - q0) lies in
+            // [0, span], one unsigned compare per entry; an empty row (lo > hi) masks them all
+            const bool full = __all_sync(0xffffffffu, (q0 >= lo) && (q0 + kBM - 1 <= hi));
+            const int vis0 = (lo <= hi) ? lo - q0 : (1 << 20);
+            const unsigned span = (lo <= hi) ? (unsigned)(hi - lo) : 0u;
             const float* ls = lse_s + buf * 128;
             const float* dl = delta_s + buf * 128;
             // P phase (needs S^T only): P^T goes to TMEM for dV; P times the cap factor stays in
@@ -397,10 +401,8 @@ __global__ void __launch_bounds__(512, 1)
                     float pp[4] = {ex2(x01.x), ex2(x01.y), ex2(x23.x), ex2(x23.y)};
                     if (!full) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int q = q0 + 32 * c + e + u;
-                            if (q < lo || q > hi) pp[u] = 0.f;
-                        }
+                        for (int u = 0; u < 4; ++u)
+                            if ((unsigned)(32 * c + e + u - vis0) > span) pp[u] = 0.f;
                     }
                     pk[e / 2] = pack_bf16x2(pp[0], pp[1]);
                     pk[e / 2 + 1] = pack_bf16x2(pp[2], pp[3]);
