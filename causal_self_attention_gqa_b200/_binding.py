@@ -33,7 +33,8 @@ EXPORTED = ["csa_workspace_size", "csa_attn_fwd", "csa_attn_bwd", "csa_device_st
             "csa_status_string", "csa_timing_enable", "csa_timing_collect", "csa_num_kernels",
             "csa_kernel_name", "csa_attn_fwd_static_scratch", "csa_selftest_bounded_wait",
             "csa_attn_bwd_after_fwd", "csa_decode_workspace_size", "csa_attn_decode",
-            "csa_prefill_workspace_size", "csa_attn_prefill"]
+            "csa_prefill_workspace_size", "csa_attn_prefill", "csa_proj_workspace_size", "csa_qkv_proj",
+            "csa_out_proj", "csa_out_proj_bwd", "csa_qkv_proj_bwd"]
 
 
 class Params(ctypes.Structure):
@@ -67,6 +68,16 @@ _lib.csa_attn_decode.argtypes = [ctypes.POINTER(Params), ctypes.c_int, _vp, _vp,
 _lib.csa_attn_decode.restype = ctypes.c_int
 _lib.csa_attn_fwd_static_scratch.argtypes = [ctypes.POINTER(Params), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.csa_attn_fwd_static_scratch.restype = ctypes.c_int
+_lib.csa_proj_workspace_size.argtypes = []
+_lib.csa_proj_workspace_size.restype = ctypes.c_size_t
+_lib.csa_qkv_proj.argtypes = [ctypes.POINTER(Params), ctypes.c_int] + [_vp] * 8 + [ctypes.c_size_t, _vp]
+_lib.csa_qkv_proj.restype = ctypes.c_int
+_lib.csa_out_proj.argtypes = [ctypes.POINTER(Params), ctypes.c_int] + [_vp] * 4 + [ctypes.c_size_t, _vp]
+_lib.csa_out_proj.restype = ctypes.c_int
+_lib.csa_out_proj_bwd.argtypes = [ctypes.POINTER(Params), ctypes.c_int] + [_vp] * 6 + [ctypes.c_size_t, _vp]
+_lib.csa_out_proj_bwd.restype = ctypes.c_int
+_lib.csa_qkv_proj_bwd.argtypes = [ctypes.POINTER(Params), ctypes.c_int] + [_vp] * 12 + [ctypes.c_size_t, _vp]
+_lib.csa_qkv_proj_bwd.restype = ctypes.c_int
 _lib.csa_selftest_bounded_wait.argtypes = [_vp, ctypes.c_size_t, _vp]
 _lib.csa_selftest_bounded_wait.restype = ctypes.c_int
 _lib.csa_device_status.argtypes = [_vp, _vp]
@@ -257,6 +268,109 @@ def attn_decode(q, k_cache, v_cache, *, causal=True, window=0, softcap=0.0, rope
     if rc != CSA_OK:
         raise CsaError(rc, "csa_attn_decode")
     return o, lse
+
+
+# ------------------------------------------------------------------ projections around attention
+def _check_f32(name, t, shape):
+    if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name} must be a contiguous CUDA fp32 tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _proj_ws(workspace, device):
+    if workspace is None:
+        workspace = torch.zeros(int(_lib.csa_proj_workspace_size()), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def _proj_shapes(x_shape, wq, wk):
+    B, T, C = x_shape
+    _, Hq, D = wq.shape
+    return B, T, C, Hq, wk.shape[1], D
+
+
+def qkv_proj(x, wq, wk, wv, *, q=None, k=None, v=None, workspace=None, stream=None):
+    """csa_qkv_proj: q = x wq, k = x wk, v = x wv (one launch); x [B,T,C], wq [C,Hq,D],
+    wk / wv [C,Hkv,D], all bf16."""
+    B, T, C, Hq, Hkv, D = _proj_shapes(x.shape, wq, wk)
+    _check_bf16("x", x, (B, T, C))
+    _check_bf16("wq", wq, (C, Hq, D))
+    _check_bf16("wk", wk, (C, Hkv, D))
+    _check_bf16("wv", wv, (C, Hkv, D))
+    q = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty((B, T, Hkv, D), dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty((B, T, Hkv, D), dtype=torch.bfloat16, device=x.device) if v is None else v
+    ws, nb = _proj_ws(workspace, x.device)
+    p = make_params(B, T, Hq, Hkv, D)
+    rc = _lib.csa_qkv_proj(ctypes.byref(p), C, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(q), _ptr(k), _ptr(v),
+                           _ptr(ws), nb, _stream(stream))
+    if rc != CSA_OK:
+        raise CsaError(rc, "csa_qkv_proj")
+    return q, k, v
+
+
+def out_proj(o, wo, *, y=None, workspace=None, stream=None):
+    """csa_out_proj: y = o wo; o [B,T,Hq,D], wo [Hq,D,C] bf16 -> y [B,T,C] bf16."""
+    B, T, Hq, D = o.shape
+    C = wo.shape[2]
+    _check_bf16("o", o, (B, T, Hq, D))
+    _check_bf16("wo", wo, (Hq, D, C))
+    y = torch.empty((B, T, C), dtype=torch.bfloat16, device=o.device) if y is None else y
+    ws, nb = _proj_ws(workspace, o.device)
+    p = make_params(B, T, Hq, Hq, D)
+    rc = _lib.csa_out_proj(ctypes.byref(p), C, _ptr(o), _ptr(wo), _ptr(y), _ptr(ws), nb, _stream(stream))
+    if rc != CSA_OK:
+        raise CsaError(rc, "csa_out_proj")
+    return y
+
+
+def out_proj_bwd(o, wo, dy, *, dout=None, dwo=None, weight_grad=True, workspace=None, stream=None):
+    """csa_out_proj_bwd: dout = dy wo^T (bf16) and, when weight_grad, dwo += o^T dy (fp32;
+    a zeroed tensor is allocated when dwo is None)."""
+    B, T, Hq, D = o.shape
+    C = wo.shape[2]
+    _check_bf16("o", o, (B, T, Hq, D))
+    _check_bf16("wo", wo, (Hq, D, C))
+    _check_bf16("dy", dy, (B, T, C))
+    dout = torch.empty_like(o) if dout is None else dout
+    if weight_grad:
+        dwo = torch.zeros((Hq, D, C), dtype=torch.float32, device=o.device) if dwo is None else dwo
+        _check_f32("dwo", dwo, (Hq, D, C))
+    else:
+        dwo = None
+    ws, nb = _proj_ws(workspace, o.device)
+    p = make_params(B, T, Hq, Hq, D)
+    rc = _lib.csa_out_proj_bwd(ctypes.byref(p), C, _ptr(o), _ptr(wo), _ptr(dy), _ptr(dout), _ptr(dwo), _ptr(ws), nb,
+                               _stream(stream))
+    if rc != CSA_OK:
+        raise CsaError(rc, "csa_out_proj_bwd")
+    return dout, dwo
+
+
+def qkv_proj_bwd(x, wq, wk, wv, dq, dk, dv, *, dx=None, dwq=None, dwk=None, dwv=None, weight_grad=True,
+                 workspace=None, stream=None):
+    """csa_qkv_proj_bwd: dx = dq wq^T + dk wk^T + dv wv^T (bf16) and, when weight_grad,
+    dwq += x^T dq, dwk += x^T dk, dwv += x^T dv (fp32; zeroed tensors allocated when None)."""
+    B, T, C, Hq, Hkv, D = _proj_shapes(x.shape, wq, wk)
+    _check_bf16("x", x, (B, T, C))
+    for name, t, shp in (("wq", wq, (C, Hq, D)), ("wk", wk, (C, Hkv, D)), ("wv", wv, (C, Hkv, D)),
+                         ("dq", dq, (B, T, Hq, D)), ("dk", dk, (B, T, Hkv, D)), ("dv", dv, (B, T, Hkv, D))):
+        _check_bf16(name, t, shp)
+    dx = torch.empty_like(x) if dx is None else dx
+    if weight_grad:
+        z = lambda t, H: torch.zeros((C, H, D), dtype=torch.float32, device=x.device) if t is None else t  # noqa: E731
+        dwq, dwk, dwv = z(dwq, Hq), z(dwk, Hkv), z(dwv, Hkv)
+        for name, t, H in (("dwq", dwq, Hq), ("dwk", dwk, Hkv), ("dwv", dwv, Hkv)):
+            _check_f32(name, t, (C, H, D))
+    else:
+        dwq = dwk = dwv = None
+    ws, nb = _proj_ws(workspace, x.device)
+    p = make_params(B, T, Hq, Hkv, D)
+    rc = _lib.csa_qkv_proj_bwd(ctypes.byref(p), C, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(dx), _ptr(dwq), _ptr(dwk), _ptr(dwv), _ptr(ws), nb, _stream(stream))
+    if rc != CSA_OK:
+        raise CsaError(rc, "csa_qkv_proj_bwd")
+    return dx, dwq, dwk, dwv
 
 
 def device_status(workspace, stream=None) -> int:

@@ -6,6 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <initializer_list>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -529,6 +530,274 @@ int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_ca
     return timed(kDecode, st, [&] { return launch_decode(P, d, q, tk, tv, part, done, o, lse, st); });
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------------ projections around attention
+// x [B*T, C] -> q, k, v through the 3-D weights, o -> y through wo, and the backward products
+// (gemm.cu).  Every matrix is row-major; the status word sits at the start of the workspace.
+namespace csa {
+cudaError_t launch_gemm(const GemmMaps& maps, const GemmArgs& g, cudaStream_t st);
+namespace {
+
+// Row-major [rows, cols] matrix (bf16, or fp32 when f32), boxes of box_cols x box_rows
+// elements with 128-byte swizzle (box_cols x element size = 128 bytes).
+bool make_map_2d(CUtensorMap* m, const void* base, long long rows, int cols, bool f32, int box_cols,
+                 int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int es = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * es};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Tile width.  Pieced N (npieces > 1): the widest of 256, 192, 128, 64 that divides every
+// piece.  One piece: the one that leaves the fewest unused columns in the last tile (ties go
+// to the wider tile).
+int pick_bn(const int* widths, int npieces) {
+    static const int cand[4] = {256, 192, 128, 64};
+    if (npieces > 1) {
+        for (int c : cand) {
+            bool ok = true;
+            for (int i = 0; i < npieces; ++i) ok = ok && (widths[i] % c == 0);
+            if (ok) return c;
+        }
+        return 0;
+    }
+    int best = 0, waste = 1 << 30;
+    for (int c : cand) {
+        const int w = (widths[0] + c - 1) / c * c - widths[0];
+        if (w < waste) {
+            waste = w;
+            best = c;
+        }
+    }
+    return best;
+}
+
+// Fills the piece bounds (from the piece widths) and the tile / split plan.  Weight gradients
+// (split_k) cut K so that about one unit runs per SM, keeping at least 4 K blocks a split.
+void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const int* kw, int nk, bool split_k,
+               int* status) {
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.n_bound[0] = g.k_bound[0] = 0;
+    for (int i = 1; i < 4; ++i) {
+        g.n_bound[i] = (i <= nn - 1) ? g.n_bound[i - 1] + nw[i - 1] : N;
+        g.k_bound[i] = (i <= nk - 1) ? g.k_bound[i - 1] + kw[i - 1] : K;
+    }
+    g.bn = pick_bn(nw, nn);
+    g.mt = (M + 127) / 128;
+    g.nt = (N + g.bn - 1) / g.bn;
+    g.kb_total = (K + 63) / 64;
+    int splits = 1;
+    if (split_k) {
+        const int tiles = g.mt * g.nt;
+        splits = num_sms() / tiles;
+        if (splits > g.kb_total / 4) splits = g.kb_total / 4;
+        if (splits < 1) splits = 1;
+    }
+    g.kb_per_split = (g.kb_total + splits - 1) / splits;
+    g.splits = (g.kb_total + g.kb_per_split - 1) / g.kb_per_split;
+    g.units = g.mt * g.nt * g.splits;
+    g.status = status;
+}
+
+// Host-side checks shared by the projection calls: the attention parameters (for Hq, Hkv,
+// D), the model width, the piece alignment, the workspace (status word only).
+int check_proj(const csa_params* p, int d_model, const void* workspace, size_t workspace_bytes) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (d_model < 64 || d_model % 64 != 0 || d_model > (1 << 16)) return CSA_ERR_INVALID_ARG;
+    if ((p->Hkv * p->D) % 64 != 0) return CSA_ERR_INVALID_ARG;
+    if (!workspace) return CSA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return CSA_ERR_ALIGNMENT;
+    if (workspace_bytes < kAlign) return CSA_ERR_WORKSPACE;
+    return CSA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ptrs) {
+    for (const void* q : ptrs)
+        if (!q) return CSA_ERR_INVALID_ARG;
+    for (const void* q : ptrs)
+        if (!aligned(q, 16)) return CSA_ERR_ALIGNMENT;
+    return CSA_OK;
+}
+
+int run_gemm(int kernel, const GemmMaps& maps, const GemmArgs& g, cudaStream_t st) {
+    if (g.units == 0) return CSA_OK;
+    return timed(kernel, st, [&] { return launch_gemm(maps, g, st); });
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" {
+
+size_t csa_proj_workspace_size(void) { return kAlign; }
+
+int csa_qkv_proj(const csa_params* p, int d_model, const void* x, const void* wq, const void* wk, const void* wv,
+                 void* q, void* k, void* v, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_proj(p, d_model, workspace, workspace_bytes);
+    if (rc) return rc;
+    if ((rc = check_ptrs({x, wq, wk, wv, q, k, v}))) return rc;
+    if ((rc = check_device())) return rc;
+    const long long M = (long long)p->B * p->T;
+    if (M == 0) return CSA_OK;
+    const int hq = p->Hq * p->D, hk = p->Hkv * p->D;
+    const int nw[3] = {hq, hk, hk};
+    GemmArgs g{};
+    g.a_mn = 0;
+    g.b_mn = 1;
+    g.f32_out = 0;
+    g.b_by_k = 0;
+    plan_gemm(g, (int)M, hq + 2 * hk, d_model, nw, 3, nullptr, 1, false, static_cast<int*>(workspace));
+    GemmMaps maps;
+    const void* w3[3] = {wq, wk, wv};
+    void* o3[3] = {q, k, v};
+    bool ok = make_map_2d(&maps.a[0], x, M, d_model, false, 64, 128);
+    maps.a[1] = maps.a[2] = maps.a[0];
+    for (int i = 0; i < 3; ++i) {
+        ok = ok && make_map_2d(&maps.b[i], w3[i], d_model, nw[i], false, 64, 64);
+        ok = ok && make_map_2d(&maps.c[i], o3[i], M, nw[i], false, 64, 32);
+    }
+    if (!ok) return CSA_ERR_CUDA;
+    return run_gemm(kGemmQkv, maps, g, static_cast<cudaStream_t>(stream));
+}
+
+int csa_out_proj(const csa_params* p, int d_model, const void* o, const void* wo, void* y, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    int rc = check_proj(p, d_model, workspace, workspace_bytes);
+    if (rc) return rc;
+    if ((rc = check_ptrs({o, wo, y}))) return rc;
+    if ((rc = check_device())) return rc;
+    const long long M = (long long)p->B * p->T;
+    if (M == 0) return CSA_OK;
+    const int hq = p->Hq * p->D;
+    GemmArgs g{};
+    g.a_mn = 0;
+    g.b_mn = 1;
+    g.f32_out = 0;
+    g.b_by_k = 0;
+    plan_gemm(g, (int)M, d_model, hq, &d_model, 1, nullptr, 1, false, static_cast<int*>(workspace));
+    GemmMaps maps;
+    bool ok = make_map_2d(&maps.a[0], o, M, hq, false, 64, 128) && make_map_2d(&maps.b[0], wo, hq, d_model, false, 64, 64) &&
+              make_map_2d(&maps.c[0], y, M, d_model, false, 64, 32);
+    if (!ok) return CSA_ERR_CUDA;
+    maps.a[1] = maps.a[2] = maps.a[0];
+    maps.b[1] = maps.b[2] = maps.b[0];
+    maps.c[1] = maps.c[2] = maps.c[0];
+    return run_gemm(kGemmOut, maps, g, static_cast<cudaStream_t>(stream));
+}
+
+int csa_out_proj_bwd(const csa_params* p, int d_model, const void* o, const void* wo, const void* dy, void* dout,
+                     float* dwo, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_proj(p, d_model, workspace, workspace_bytes);
+    if (rc) return rc;
+    if ((rc = check_ptrs({o, wo, dy, dout}))) return rc;
+    if (dwo && !aligned(dwo, 16)) return CSA_ERR_ALIGNMENT;
+    if ((rc = check_device())) return rc;
+    const long long M = (long long)p->B * p->T;
+    if (M == 0) return CSA_OK;
+    const int hq = p->Hq * p->D;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(workspace);
+    {  // dout = dy wo^T: A = dy [M, C] K-major, B = wo [hq, C] K-major
+        GemmArgs g{};
+        g.a_mn = 0;
+        g.b_mn = 0;
+        g.f32_out = 0;
+        g.b_by_k = 0;
+        plan_gemm(g, (int)M, hq, d_model, &hq, 1, nullptr, 1, false, status);
+        GemmMaps maps;
+        bool ok = make_map_2d(&maps.a[0], dy, M, d_model, false, 64, 128) &&
+                  make_map_2d(&maps.b[0], wo, hq, d_model, false, 64, g.bn) &&
+                  make_map_2d(&maps.c[0], dout, M, hq, false, 64, 32);
+        if (!ok) return CSA_ERR_CUDA;
+        maps.a[1] = maps.a[2] = maps.a[0];
+        maps.b[1] = maps.b[2] = maps.b[0];
+        maps.c[1] = maps.c[2] = maps.c[0];
+        if ((rc = run_gemm(kGemmDout, maps, g, st))) return rc;
+    }
+    if (!dwo) return CSA_OK;
+    // dwo += o^T dy: A = o [M, hq] read M-major, B = dy [M, C] N-major, fp32 reduce-adds
+    GemmArgs g{};
+    g.a_mn = 1;
+    g.b_mn = 1;
+    g.f32_out = 1;
+    g.b_by_k = 0;
+    plan_gemm(g, hq, d_model, (int)M, &d_model, 1, nullptr, 1, true, status);
+    GemmMaps maps;
+    bool ok = make_map_2d(&maps.a[0], o, M, hq, false, 64, 64) && make_map_2d(&maps.b[0], dy, M, d_model, false, 64, 64) &&
+              make_map_2d(&maps.c[0], dwo, hq, d_model, true, 32, 32);
+    if (!ok) return CSA_ERR_CUDA;
+    maps.a[1] = maps.a[2] = maps.a[0];
+    maps.b[1] = maps.b[2] = maps.b[0];
+    maps.c[1] = maps.c[2] = maps.c[0];
+    return run_gemm(kGemmDwo, maps, g, st);
+}
+
+int csa_qkv_proj_bwd(const csa_params* p, int d_model, const void* x, const void* wq, const void* wk, const void* wv,
+                     const void* dq, const void* dk, const void* dv, void* dx, float* dwq, float* dwk, float* dwv,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_proj(p, d_model, workspace, workspace_bytes);
+    if (rc) return rc;
+    if ((rc = check_ptrs({x, wq, wk, wv, dq, dk, dv, dx}))) return rc;
+    const bool wgrad = dwq || dwk || dwv;
+    if (wgrad && (rc = check_ptrs({dwq, dwk, dwv}))) return rc;
+    if ((rc = check_device())) return rc;
+    const long long M = (long long)p->B * p->T;
+    if (M == 0) return CSA_OK;
+    const int hq = p->Hq * p->D, hk = p->Hkv * p->D;
+    const int w3[3] = {hq, hk, hk};
+    const void* wt[3] = {wq, wk, wv};
+    const void* gt[3] = {dq, dk, dv};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(workspace);
+    {  // dx = dq wq^T + dk wk^T + dv wv^T: K pieced; A = dq|dk|dv K-major, B = wq|wk|wv [C, h] K-major
+        GemmArgs g{};
+        g.a_mn = 0;
+        g.b_mn = 0;
+        g.f32_out = 0;
+        g.b_by_k = 1;
+        plan_gemm(g, (int)M, d_model, hq + 2 * hk, &d_model, 1, w3, 3, false, status);
+        GemmMaps maps;
+        bool ok = make_map_2d(&maps.c[0], dx, M, d_model, false, 64, 32);
+        for (int i = 0; i < 3; ++i) {
+            ok = ok && make_map_2d(&maps.a[i], gt[i], M, w3[i], false, 64, 128);
+            ok = ok && make_map_2d(&maps.b[i], wt[i], d_model, w3[i], false, 64, g.bn);
+        }
+        if (!ok) return CSA_ERR_CUDA;
+        maps.c[1] = maps.c[2] = maps.c[0];
+        if ((rc = run_gemm(kGemmDx, maps, g, st))) return rc;
+    }
+    if (!wgrad) return CSA_OK;
+    // dwq|dwk|dwv += x^T [dq|dk|dv]: A = x [M, C] read M-major, B and C pieced by N, fp32
+    GemmArgs g{};
+    g.a_mn = 1;
+    g.b_mn = 1;
+    g.f32_out = 1;
+    g.b_by_k = 0;
+    plan_gemm(g, d_model, hq + 2 * hk, (int)M, w3, 3, nullptr, 1, true, status);
+    GemmMaps maps;
+    float* dw3[3] = {dwq, dwk, dwv};
+    bool ok = make_map_2d(&maps.a[0], x, M, d_model, false, 64, 64);
+    maps.a[1] = maps.a[2] = maps.a[0];
+    for (int i = 0; i < 3; ++i) {
+        ok = ok && make_map_2d(&maps.b[i], gt[i], M, w3[i], false, 64, 64);
+        ok = ok && make_map_2d(&maps.c[i], dw3[i], d_model, w3[i], true, 32, 32);
+    }
+    if (!ok) return CSA_ERR_CUDA;
+    return run_gemm(kGemmDw, maps, g, st);
+}
+
 int csa_selftest_bounded_wait(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace) return CSA_ERR_INVALID_ARG;
     if (!aligned(workspace, 256)) return CSA_ERR_ALIGNMENT;
@@ -607,7 +876,9 @@ int csa_num_kernels(void) { return kNumKernels; }
 const char* csa_kernel_name(int k) {
     static const char* names[kNumKernels] = {"k_prep",          "k_qk_prologue", "k_attn_fwd",
                                              "k_bwd_pre",       "k_attn_bwd",    "k_grad_finalize",
-                                             "k_decode"};
+                                             "k_decode",        "k_gemm_qkv",    "k_gemm_out",
+                                             "k_gemm_dout",     "k_gemm_dwo",    "k_gemm_dx",
+                                             "k_gemm_dw"};
     return (k >= 0 && k < kNumKernels) ? names[k] : "";
 }
 

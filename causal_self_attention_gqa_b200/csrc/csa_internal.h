@@ -4,6 +4,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "csa.h"
@@ -82,6 +83,25 @@ struct DecodePlan {
     size_t part_bytes, done_bytes;
 };
 
+// One projection GEMM (gemm.cu): C[M, N] = sum_k A[m, k] B[k, n] over row-major bf16
+// matrices, fp32 accumulation; C is bf16 (stored) or fp32 (added to what C holds).  A is read
+// K-major ([M, K] in memory) or M-major ([K, M]); B K-major ([N, K]) or N-major ([K, N]).
+// An operand may come in up to three pieces (separate tensors, one tensor map each): pieces
+// of C, and of B when b_by_k is 0, split N at n_bound; pieces of A, and of B when b_by_k is
+// 1, split K at k_bound.  Unused bounds equal N (resp. K).
+struct GemmArgs {
+    int M, N, K;
+    int bn;                 // N per tile: 64, 128, 192 or 256 (divides every inner N bound)
+    int a_mn, b_mn, f32_out;
+    int b_by_k;
+    int n_bound[4], k_bound[4];  // [0] = 0, [3] = N (resp. K); inner bounds multiples of bn (64)
+    int mt, nt, splits, kb_total, kb_per_split, units;
+    int* status;
+};
+struct GemmMaps {
+    CUtensorMap a[3], b[3], c[3];
+};
+
 // Streaming multiprocessors of the current device (cached per device).
 int num_sms();
 
@@ -92,7 +112,8 @@ cudaError_t ensure_dyn_smem(const void* kernel, int bytes);
 
 // Kernel ids for the timing interface (order = csa_kernel_name()).
 enum KernelId {
-    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecode, kNumKernels
+    kPrep = 0, kPrologue, kFwd, kBwdPre, kBwd, kGradFinalize, kDecode,
+    kGemmQkv, kGemmOut, kGemmDout, kGemmDwo, kGemmDx, kGemmDw, kNumKernels
 };
 
 }  // namespace csa

@@ -147,3 +147,39 @@ def make_decode_inputs(w: DecodeWorkload) -> dict:
     kc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
     vc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
     return dict(q=q, k_cache=kc, v_cache=vc)
+
+
+# The attention layer with its projections (x -> q, k, v -> attention -> y): the attention
+# workload's shape plus the model width C.  Weights are drawn like a fan-in initialisation,
+# N(0, 1/fan_in), so that q, k, v and y have about unit variance when x does.
+@dataclass(frozen=True)
+class LayerWorkload:
+    name: str
+    attn: Workload
+    C: int
+    seed: int = 0
+
+
+LAYER_WORKLOADS = [
+    LayerWorkload("layer_gpt181m_C768_gqa8x4_T2048_D96_rope_qknorm", WORKLOADS[3], C=768, seed=1100),
+    LayerWorkload("layer_depth12_C768_gqa6x3_T2048_D128_rope_qknorm_cap50", WORKLOADS[2], C=768, seed=1101),
+]
+
+
+def make_layer_inputs(w: LayerWorkload) -> dict:
+    """bf16 CPU tensors x [B,T,C], wq [C,Hq,D], wk / wv [C,Hkv,D], wo [Hq,D,C], dy [B,T,C]."""
+    a = w.attn
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+
+    def draw(shape, std):
+        return (torch.randn(shape, generator=g, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    return dict(
+        x=draw((a.B, a.T, w.C), 1.0),
+        wq=draw((w.C, a.Hq, a.D), w.C ** -0.5),
+        wk=draw((w.C, a.Hkv, a.D), w.C ** -0.5),
+        wv=draw((w.C, a.Hkv, a.D), w.C ** -0.5),
+        wo=draw((a.Hq, a.D, w.C), (a.Hq * a.D) ** -0.5),
+        dy=draw((a.B, a.T, w.C), 1.0),
+    )

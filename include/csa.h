@@ -148,6 +148,44 @@ int csa_attn_decode(const csa_params* p, int Tq, const void* q, const void* k_ca
                     const void* v_cache, void* o, float* lse, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Projections around attention (the nanogpt-jax-181m model card, section "Architecture":
+ * 3-D attention weights wq, wk, wv of shape (d_emb, heads, head_dim) and wo of shape
+ * (heads, head_dim, d_emb); the GPT-pretraining page, section "Multihead Attention": q, k, v
+ * are linear maps of the block input x, and the attention output goes through an output
+ * projection).  No bias: the 3-D weights of the model card carry none.  With C = d_model:
+ *   x, y, dx, dy   [B, T, C] bf16
+ *   wq             [C, Hq, D] bf16;   wk, wv [C, Hkv, D] bf16;   wo [Hq, D, C] bf16
+ *   q = x wq, k = x wk, v = x wv      (sum over C; q [B,T,Hq,D], k, v [B,T,Hkv,D] bf16)
+ *   y = o wo                           (sum over heads and D; o [B,T,Hq,D])
+ * Backward, for a loss L with dy = dL/dy (and dq, dk, dv = dL/dq, ...):
+ *   csa_out_proj_bwd:  dout = dy wo^T (bf16 [B,T,Hq,D]);  dwo += o^T dy
+ *   csa_qkv_proj_bwd:  dx = dq wq^T + dk wk^T + dv wv^T (bf16);
+ *                      dwq += x^T dq, dwk += x^T dk, dwv += x^T dv
+ * Weight gradients are fp32 tensors of the weights' shapes, ADDED to what they hold (zero
+ * them for a plain gradient; leave them for accumulation over micro-batches).  Pass NULL for
+ * dwo, or for all three of dwq, dwk, dwv, to skip them.  Products accumulate in fp32; bf16
+ * outputs are rounded once, to nearest even.
+ * Requirements (CSA_ERR_INVALID_ARG otherwise): *p valid as for csa_attn_fwd (only B, T, Hq,
+ * Hkv, D are used), C a multiple of 64 (at most 65536), Hkv * D a multiple of 64.  Device
+ * pointers 16-byte aligned, caller-owned.  The workspace holds only the status word: at least
+ * csa_proj_workspace_size() bytes, 256-byte aligned (an attention workspace serves).  A
+ * bounded wait that runs out records CSA_ERR_DEVICE_TIMEOUT there, read back with
+ * csa_device_status(); these calls do not clear the word.  One launch per product: two for
+ * each backward call with weight gradients. */
+size_t csa_proj_workspace_size(void);
+int csa_qkv_proj(const csa_params* p, int d_model, const void* x, const void* wq, const void* wk,
+                 const void* wv, void* q, void* k, void* v, void* workspace, size_t workspace_bytes,
+                 void* stream);
+int csa_out_proj(const csa_params* p, int d_model, const void* o, const void* wo, void* y,
+                 void* workspace, size_t workspace_bytes, void* stream);
+int csa_out_proj_bwd(const csa_params* p, int d_model, const void* o, const void* wo,
+                     const void* dy, void* dout, float* dwo, void* workspace,
+                     size_t workspace_bytes, void* stream);
+int csa_qkv_proj_bwd(const csa_params* p, int d_model, const void* x, const void* wq,
+                     const void* wk, const void* wv, const void* dq, const void* dk,
+                     const void* dv, void* dx, float* dwq, float* dwk, float* dwv,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last call that used it (CSA_OK, CSA_ERR_DEVICE_TIMEOUT, or CSA_ERR_CUDA when the
  * synchronisation itself failed).  Resets the recorded status to CSA_OK. */

@@ -102,7 +102,40 @@ def test_status_strings(b):
         assert b.status_string(code)
     assert b.status_string(6) == "a bounded wait inside a kernel ran out"
     assert b.kernel_names() == ["k_prep", "k_qk_prologue", "k_attn_fwd", "k_bwd_pre", "k_attn_bwd",
-                                "k_grad_finalize", "k_decode"]
+                                "k_grad_finalize", "k_decode", "k_gemm_qkv", "k_gemm_out", "k_gemm_dout",
+                                "k_gemm_dwo", "k_gemm_dx", "k_gemm_dw"]
+
+
+def test_projection_arguments_are_checked_on_the_host(b):
+    """csa_qkv_proj / csa_out_proj / csa_out_proj_bwd / csa_qkv_proj_bwd: model width, piece
+    alignment, pointers and workspace are rejected before anything is enqueued (fake
+    pointers: every call here fails a check)."""
+    lib = b.lib
+    good = b.make_params(2, 128, 8, 4, 96)
+    assert lib.csa_proj_workspace_size() == 256
+    P = [0x1000 * (i + 1) for i in range(12)]
+    ws = 0x100000
+
+    def qkv(p, C, ptrs=P, w=ws, n=256):
+        return lib.csa_qkv_proj(ctypes.byref(p), C, *ptrs[:7], w, n, None)
+
+    assert qkv(good, 96) == b.CSA_ERR_INVALID_ARG        # C not a multiple of 64
+    assert qkv(good, 0) == b.CSA_ERR_INVALID_ARG
+    assert qkv(b.make_params(2, 128, 2, 1, 32), 128) == b.CSA_ERR_INVALID_ARG  # Hkv * D = 32
+    assert qkv(b.make_params(2, 128, 6, 4, 64), 128) == b.CSA_ERR_INVALID_ARG  # Hq % Hkv != 0
+    assert qkv(good, 768, w=None) == b.CSA_ERR_INVALID_ARG
+    assert qkv(good, 768, w=ws + 16) == b.CSA_ERR_ALIGNMENT
+    assert qkv(good, 768, n=128) == b.CSA_ERR_WORKSPACE
+    bad = list(P)
+    bad[3] = 0x4008  # wv misaligned
+    assert qkv(good, 768, ptrs=bad) == b.CSA_ERR_ALIGNMENT
+    bad[3] = 0
+    assert qkv(good, 768, ptrs=bad) == b.CSA_ERR_INVALID_ARG
+    assert lib.csa_out_proj(ctypes.byref(good), 100, *P[:3], ws, 256, None) == b.CSA_ERR_INVALID_ARG
+    assert lib.csa_out_proj(ctypes.byref(good), 768, P[0], 0, P[2], ws, 256, None) == b.CSA_ERR_INVALID_ARG
+    assert lib.csa_out_proj_bwd(ctypes.byref(good), 768, *P[:4], 0x5004, ws, 256, None) == b.CSA_ERR_ALIGNMENT
+    assert lib.csa_qkv_proj_bwd(ctypes.byref(good), 768, *P[:8], P[8], 0, P[10], ws, 256,
+                                None) == b.CSA_ERR_INVALID_ARG  # dwk missing while dwq is given
 
 
 def test_decode_arguments_are_checked_on_the_host(b):
