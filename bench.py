@@ -43,8 +43,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from causal_self_attention_gqa_b200.workloads import (BY_NAME, DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
-                                                      make_decode_inputs, make_inputs)
+from causal_self_attention_gqa_b200.workloads import (BY_NAME, DECODE_WORKLOADS, LAYER_WORKLOADS,  # noqa: E402
+                                                      WORKLOADS, LayerWorkload, make_decode_inputs, make_inputs)
 
 DEFAULT_WORKLOAD = WORKLOADS[3].name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -467,6 +467,98 @@ def measure_training(w, dev, steps: int, warmup: int, flush) -> dict:
             "kernels": {n: {"ms_avg": t / c, "share": t / tot_k} for n, (t, c) in kt.items()}}
 
 
+GEMM_KERNELS = ("k_gemm_qkv", "k_gemm_out", "k_gemm_dout", "k_gemm_dwo", "k_gemm_dx", "k_gemm_dw")
+
+
+def gemm_flops(lw) -> dict:
+    """Multiply-adds x 2 of each projection product of one layer step (M = B*T tokens)."""
+    a = lw.attn
+    M, C, hq, hk = a.B * a.T, lw.C, a.Hq * a.D, a.Hkv * a.D
+    qkv = 2.0 * M * C * (hq + 2 * hk)
+    out = 2.0 * M * hq * C
+    return {"k_gemm_qkv": qkv, "k_gemm_out": out, "k_gemm_dout": out, "k_gemm_dwo": out, "k_gemm_dx": qkv,
+            "k_gemm_dw": qkv}
+
+
+def measure_layer(lw, dev, steps: int, warmup: int, flush) -> dict:
+    """The attention layer's training step with its projections, 1 GPU: csa_qkv_proj,
+    csa_attn_fwd, csa_out_proj, then csa_out_proj_bwd (with dwo), csa_attn_bwd_after_fwd and
+    csa_qkv_proj_bwd (with dwq, dwk, dwv).  Timed like the headline (per-step events, L2
+    flushed between steps outside them); TFLOP/s counts the attention's algorithmic FLOPs plus
+    2 per multiply-add of the six projection products.  Weight gradients accumulate over the
+    steps (the calls add into them), as under gradient accumulation."""
+    from causal_self_attention_gqa_b200 import _binding as csa
+    from causal_self_attention_gqa_b200.workloads import make_layer_inputs
+    a = lw.attn
+    inp = make_layer_inputs(lw)
+    f_fwd, f_bwd, _ = flops(a, None)
+    gf = gemm_flops(lw)
+    kw = a.options()
+    x, wq, wk, wv, wo, dy = (inp[n].to(dev) for n in ("x", "wq", "wk", "wv", "wo", "dy"))
+    q = torch.empty((a.B, a.T, a.Hq, a.D), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((a.B, a.T, a.Hkv, a.D), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    o, dout, dq = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dk, dv = torch.empty_like(k), torch.empty_like(k)
+    y, dx = torch.empty_like(x), torch.empty_like(x)
+    lse = torch.empty((a.B, a.Hq, a.T), dtype=torch.float32, device=dev)
+    dwq, dwk, dwv = (torch.zeros(t.shape, dtype=torch.float32, device=dev) for t in (wq, wk, wv))
+    dwo = torch.zeros(wo.shape, dtype=torch.float32, device=dev)
+    ws = csa.workspace_for(q, k, True, **kw)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.qkv_proj(x, wq, wk, wv, q=q, k=k, v=v, workspace=ws)
+        csa.attn_fwd(q, k, v, out=o, lse=lse, workspace=ws, **kw)
+        csa.out_proj(o, wo, y=y, workspace=ws)
+        csa.out_proj_bwd(o, wo, dy, dout=dout, dwo=dwo, workspace=ws)
+        csa.attn_bwd(q, k, v, o, dout, lse, dq=dq, dk=dk, dv=dv, workspace=ws, after_fwd=True, **kw)
+        csa.qkv_proj_bwd(x, wq, wk, wv, dq, dk, dv, dx=dx, dwq=dwq, dwk=dwk, dwv=dwv, workspace=ws)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"{lw.name}: device status after warm-up: {csa.status_string(rc)}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    csa.timing_enable(True)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    csa.timing_enable(False)
+    kt = {n: tc for n, tc in csa.timing_collect().items() if tc[1] > 0}
+    rc = csa.device_status(ws)
+    if rc != 0:
+        raise RuntimeError(f"{lw.name}: device status after the timed steps: {csa.status_string(rc)}")
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tot_k = sum(t for t, _ in kt.values()) or 1.0
+    gemm = {}
+    for n in GEMM_KERNELS:
+        t, c = kt[n]
+        tf = gf[n] / (t / c * 1e-3) / 1e12
+        gemm[n] = {"ms_avg": t / c, "tflops": tf, "frac_of_measured_burst": tf / peak, "flops": gf[n]}
+    g_ms = sum(kt[n][0] for n in GEMM_KERNELS) / steps
+    g_fl = sum(gf.values())
+    top = max(GEMM_KERNELS, key=lambda n: kt[n][0])
+    return {"ms_per_step": ms, "tflops": (f_fwd + f_bwd + g_fl) / (ms * 1e-3) / 1e12,
+            "tokens_per_s": a.B * a.T / (ms * 1e-3), "flops_per_step": f_fwd + f_bwd + g_fl,
+            "projection_flops_per_step": g_fl, "projection_ms_per_step": g_ms,
+            "projection_tflops": g_fl / (g_ms * 1e-3) / 1e12, "gemm": gemm,
+            "roofline": {"bound": "tensor", "achieved": gemm[top]["tflops"], "peak": peak, "unit": "TFLOP/s",
+                         "frac": gemm[top]["tflops"] / peak, "traffic": None, "kernel": top,
+                         "peak_source": f"{src}, bf16_tflops"},
+            "config": {"workload": lw.name, "B": a.B, "T": a.T, "C": lw.C, "Hq": a.Hq, "Hkv": a.Hkv, "D": a.D,
+                       "options": kw},
+            "steps": steps, "warmup": max(warmup, 3), "launches_per_step": sum(c for _, c in kt.values()) / steps,
+            "kernels": {n: {"ms_avg": t / c, "share": t / tot_k} for n, (t, c) in kt.items()}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,6 +573,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling cases)")
     ap.add_argument("--prefill", action="store_true",
                     help="time the forward over a KV cache (csa_attn_prefill) instead of the training step")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the attention layer with its projections (181M shape, C = 768) instead")
     ap.add_argument("--decode", action="store_true",
                     help="time the KV-cache decode step (csa_attn_decode) instead of the training step")
     ap.add_argument("--profile-step", action="store_true",
@@ -491,6 +585,17 @@ def main():
         w = w.with_(B=args.batch)
     if args.profile_step:
         return profile_step(w)
+    if args.layer:
+        lw = LAYER_WORKLOADS[0]
+        if args.batch:
+            lw = LayerWorkload(lw.name, lw.attn.with_(B=args.batch), C=lw.C, seed=lw.seed)
+        dev = torch.device("cuda:0")
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        r = measure_layer(lw, dev, args.steps, args.warmup, flush)
+        print(json.dumps({"metric": "attention layer with projections, fwd+bwd: algorithmic TFLOP/s",
+                          "value": r["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "higher_is_better": True,
+                          "dtype": "bf16", "data": "synthetic (seeded bf16; see workloads.py)", **r}))
+        return 0
     if args.decode:
         print(json.dumps(measure_decode(args.steps, args.warmup, args.batch)))
         return 0
@@ -672,6 +777,8 @@ def main():
         per_workload[pl["config"]["workload"]] = {
             "ms_per_step": pl["ms_per_step"], "tflops": pl["value"], "tokens_per_s": pl["tokens_per_s"],
             "roofline": pl["roofline"], "kernels": pl["kernels"], "steps": pl["steps"], "warmup": pl["warmup"]}
+        for lw in LAYER_WORKLOADS:
+            per_workload[lw.name] = measure_layer(lw, dev, args.steps, args.warmup, flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
