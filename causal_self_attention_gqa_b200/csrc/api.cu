@@ -557,25 +557,30 @@ bool make_map_2d(CUtensorMap* m, const void* base, long long rows, int cols, boo
     return r == CUDA_SUCCESS;
 }
 
-// Tile width.  Pieced N (npieces > 1): the widest of 256, 192, 128, 64 that divides every
-// piece.  One piece: the one that leaves the fewest unused columns in the last tile (ties go
-// to the wider tile).
-int pick_bn(const int* widths, int npieces) {
+// Tile width: one of 256, 192, 128, 64 that divides every piece of N (all four when N is one
+// piece).  The persistent grid gives each SM ceil(tiles / SMs) tiles, so the launch takes
+// about that many tile times.  A tile's time is its width plus a fixed share worth 256
+// columns -- the 128-row A operand streams through the SM whatever the width (fitted to the
+// 181M layer: 256-wide tiles in 6 waves beat 192-wide ones in 7).  The weight gradients
+// (split over K to fill the SMs) take the widest width instead.
+int pick_bn(const int* widths, int npieces, int M, bool split_k) {
     static const int cand[4] = {256, 192, 128, 64};
-    if (npieces > 1) {
-        for (int c : cand) {
-            bool ok = true;
-            for (int i = 0; i < npieces; ++i) ok = ok && (widths[i] % c == 0);
-            if (ok) return c;
-        }
-        return 0;
-    }
-    int best = 0, waste = 1 << 30;
+    int N = 0;
+    for (int i = 0; i < npieces; ++i) N += widths[i];
+    const long long mt = (M + 127) / 128;
+    const long long sms = num_sms();
+    int best = 0;
+    long long best_cost = 0;
     for (int c : cand) {
-        const int w = (widths[0] + c - 1) / c * c - widths[0];
-        if (w < waste) {
-            waste = w;
+        bool ok = true;
+        for (int i = 0; i < npieces && npieces > 1; ++i) ok = ok && (widths[i] % c == 0);
+        if (!ok) continue;
+        if (split_k) return c;
+        const long long tiles = mt * ((N + c - 1) / c);
+        const long long cost = (tiles + sms - 1) / sms * (c + 256);
+        if (best == 0 || cost < best_cost) {
             best = c;
+            best_cost = cost;
         }
     }
     return best;
@@ -593,7 +598,7 @@ void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const in
         g.n_bound[i] = (i <= nn - 1) ? g.n_bound[i - 1] + nw[i - 1] : N;
         g.k_bound[i] = (i <= nk - 1) ? g.k_bound[i - 1] + kw[i - 1] : K;
     }
-    g.bn = pick_bn(nw, nn);
+    g.bn = pick_bn(nw, nn, M, split_k);
     g.mt = (M + 127) / 128;
     g.nt = (N + g.bn - 1) / g.bn;
     g.kb_total = (K + 63) / 64;

@@ -64,13 +64,18 @@ def _rand_bf16(shape, seed, std=1.0):
 
 
 SHAPES = [
-    # (B, T, C, Hq, Hkv, D): ragged row tails, every tile width, all head dims
-    (2, 300, 256, 4, 2, 64),    # pieces 256 / 128 / 128 -> 128-wide tiles
-    (1, 200, 768, 8, 4, 96),    # 768 / 384 / 384 -> 192-wide tiles
-    (1, 130, 768, 6, 3, 128),   # 768 / 384 / 384, D = 128
+    # (B, T, C, Hq, Hkv, D): ragged row tails, all head dims, and between them every tile
+    # width of every operand form (the width follows the piece sizes and the wave count)
+    (2, 300, 256, 4, 2, 64),    # small: 64-wide bf16 tiles; dw 128-wide
+    (1, 200, 768, 8, 4, 96),    # 768 / 384 / 384 pieces; dw 192-wide
+    (1, 130, 768, 6, 3, 128),   # D = 128
     (2, 128, 192, 6, 6, 32),    # 192 / 192 / 192
-    (1, 77, 320, 2, 1, 64),     # 128 / 64 / 64 -> 64-wide tiles; fewer rows than one tile
-    (3, 700, 512, 8, 8, 64),    # 512 x 3 -> 256-wide tiles
+    (1, 77, 320, 2, 1, 64),     # 128 / 64 / 64 pieces; fewer rows than one tile; dw 64-wide
+    (3, 700, 512, 8, 8, 64),    # Q/K/V 256-wide, dw 256-wide
+    (1, 18944, 512, 8, 4, 64),  # 148 row tiles: every product 256-wide
+    (1, 18944, 640, 5, 5, 128),  # Q/K/V and dw 128-wide
+    (1, 2048, 768, 8, 4, 96),    # y, dO, dx 128-wide
+    (2, 4096, 640, 5, 5, 128),   # y, dO, dx 192-wide
 ]
 
 
