@@ -587,9 +587,13 @@ int pick_bn(const int* widths, int npieces, int M, bool split_k) {
 }
 
 // Fills the piece bounds (from the piece widths) and the tile / split plan.  Weight gradients
-// (split_k) cut K so that about one unit runs per SM, keeping at least 4 K blocks a split.
+// (split_k) cut K so that about one unit runs per SM (per CTA pair), keeping at least 4 K
+// blocks a split.  Large products run on CTA pairs (256 x 256 tiles, cta_group::2) when
+// allow_pair: at least one unit for every pair of SMs.  A K-major B with several N pieces
+// cannot (its 128-column half-box would straddle them); the callers pass allow_pair = false
+// there.
 void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const int* kw, int nk, bool split_k,
-               int* status) {
+               bool allow_pair, int* status) {
     g.M = M;
     g.N = N;
     g.K = K;
@@ -598,10 +602,32 @@ void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const in
         g.n_bound[i] = (i <= nn - 1) ? g.n_bound[i - 1] + nw[i - 1] : N;
         g.k_bound[i] = (i <= nk - 1) ? g.k_bound[i - 1] + kw[i - 1] : K;
     }
+    g.kb_total = (K + 63) / 64;
+    g.status = status;
+    const int pairs = num_sms() / 2;
+    if (allow_pair) {
+        const int mt2 = (M + 255) / 256, nt2 = (N + 255) / 256;
+        int splits = 1;
+        if (split_k) {
+            splits = pairs / (mt2 * nt2);
+            if (splits > g.kb_total / 4) splits = g.kb_total / 4;
+            if (splits < 1) splits = 1;
+        }
+        if (mt2 * nt2 * splits >= (split_k ? pairs / 2 : pairs)) {
+            g.pair = 1;
+            g.bn = 256;
+            g.mt = mt2;
+            g.nt = nt2;
+            g.kb_per_split = (g.kb_total + splits - 1) / splits;
+            g.splits = (g.kb_total + g.kb_per_split - 1) / g.kb_per_split;
+            g.units = g.mt * g.nt * g.splits;
+            return;
+        }
+    }
+    g.pair = 0;
     g.bn = pick_bn(nw, nn, M, split_k);
     g.mt = (M + 127) / 128;
     g.nt = (N + g.bn - 1) / g.bn;
-    g.kb_total = (K + 63) / 64;
     int splits = 1;
     if (split_k) {
         const int tiles = g.mt * g.nt;
@@ -612,7 +638,6 @@ void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const in
     g.kb_per_split = (g.kb_total + splits - 1) / splits;
     g.splits = (g.kb_total + g.kb_per_split - 1) / g.kb_per_split;
     g.units = g.mt * g.nt * g.splits;
-    g.status = status;
 }
 
 // Host-side checks shared by the projection calls: the attention parameters (for Hq, Hkv,
@@ -663,7 +688,7 @@ int csa_qkv_proj(const csa_params* p, int d_model, const void* x, const void* wq
     g.b_mn = 1;
     g.f32_out = 0;
     g.b_by_k = 0;
-    plan_gemm(g, (int)M, hq + 2 * hk, d_model, nw, 3, nullptr, 1, false, static_cast<int*>(workspace));
+    plan_gemm(g, (int)M, hq + 2 * hk, d_model, nw, 3, nullptr, 1, false, true, static_cast<int*>(workspace));
     GemmMaps maps;
     const void* w3[3] = {wq, wk, wv};
     void* o3[3] = {q, k, v};
@@ -691,7 +716,7 @@ int csa_out_proj(const csa_params* p, int d_model, const void* o, const void* wo
     g.b_mn = 1;
     g.f32_out = 0;
     g.b_by_k = 0;
-    plan_gemm(g, (int)M, d_model, hq, &d_model, 1, nullptr, 1, false, static_cast<int*>(workspace));
+    plan_gemm(g, (int)M, d_model, hq, &d_model, 1, nullptr, 1, false, true, static_cast<int*>(workspace));
     GemmMaps maps;
     bool ok = make_map_2d(&maps.a[0], o, M, hq, false, 64, 128) && make_map_2d(&maps.b[0], wo, hq, d_model, false, 64, 64) &&
               make_map_2d(&maps.c[0], y, M, d_model, false, 64, 32);
@@ -720,10 +745,10 @@ int csa_out_proj_bwd(const csa_params* p, int d_model, const void* o, const void
         g.b_mn = 0;
         g.f32_out = 0;
         g.b_by_k = 0;
-        plan_gemm(g, (int)M, hq, d_model, &hq, 1, nullptr, 1, false, status);
+        plan_gemm(g, (int)M, hq, d_model, &hq, 1, nullptr, 1, false, true, status);
         GemmMaps maps;
         bool ok = make_map_2d(&maps.a[0], dy, M, d_model, false, 64, 128) &&
-                  make_map_2d(&maps.b[0], wo, hq, d_model, false, 64, g.bn) &&
+                  make_map_2d(&maps.b[0], wo, hq, d_model, false, 64, g.pair ? 128 : g.bn) &&
                   make_map_2d(&maps.c[0], dout, M, hq, false, 64, 32);
         if (!ok) return CSA_ERR_CUDA;
         maps.a[1] = maps.a[2] = maps.a[0];
@@ -738,7 +763,7 @@ int csa_out_proj_bwd(const csa_params* p, int d_model, const void* o, const void
     g.b_mn = 1;
     g.f32_out = 1;
     g.b_by_k = 0;
-    plan_gemm(g, hq, d_model, (int)M, &d_model, 1, nullptr, 1, true, status);
+    plan_gemm(g, hq, d_model, (int)M, &d_model, 1, nullptr, 1, true, true, status);
     GemmMaps maps;
     bool ok = make_map_2d(&maps.a[0], o, M, hq, false, 64, 64) && make_map_2d(&maps.b[0], dy, M, d_model, false, 64, 64) &&
               make_map_2d(&maps.c[0], dwo, hq, d_model, true, 32, 32);
@@ -772,12 +797,12 @@ int csa_qkv_proj_bwd(const csa_params* p, int d_model, const void* x, const void
         g.b_mn = 0;
         g.f32_out = 0;
         g.b_by_k = 1;
-        plan_gemm(g, (int)M, d_model, hq + 2 * hk, &d_model, 1, w3, 3, false, status);
+        plan_gemm(g, (int)M, d_model, hq + 2 * hk, &d_model, 1, w3, 3, false, true, status);
         GemmMaps maps;
         bool ok = make_map_2d(&maps.c[0], dx, M, d_model, false, 64, 32);
         for (int i = 0; i < 3; ++i) {
             ok = ok && make_map_2d(&maps.a[i], gt[i], M, w3[i], false, 64, 128);
-            ok = ok && make_map_2d(&maps.b[i], wt[i], d_model, w3[i], false, 64, g.bn);
+            ok = ok && make_map_2d(&maps.b[i], wt[i], d_model, w3[i], false, 64, g.pair ? 128 : g.bn);
         }
         if (!ok) return CSA_ERR_CUDA;
         maps.c[1] = maps.c[2] = maps.c[0];
@@ -790,7 +815,7 @@ int csa_qkv_proj_bwd(const csa_params* p, int d_model, const void* x, const void
     g.b_mn = 1;
     g.f32_out = 1;
     g.b_by_k = 0;
-    plan_gemm(g, d_model, hq + 2 * hk, (int)M, w3, 3, nullptr, 1, true, status);
+    plan_gemm(g, d_model, hq + 2 * hk, (int)M, w3, 3, nullptr, 1, true, true, status);
     GemmMaps maps;
     float* dw3[3] = {dwq, dwk, dwv};
     bool ok = make_map_2d(&maps.a[0], x, M, d_model, false, 64, 64);

@@ -96,6 +96,7 @@ struct GemmArgs {
     int b_by_k;
     int n_bound[4], k_bound[4];  // [0] = 0, [3] = N (resp. K); inner bounds multiples of bn (64)
     int mt, nt, splits, kb_total, kb_per_split, units;
+    int pair;               // 1: CTA pairs (cta_group::2), 256-row x 256-column tiles, mt counts 256-row tiles
     int* status;
 };
 struct GemmMaps {
