@@ -19,7 +19,7 @@ import torch
 import oracle
 import oracle.proj as proj
 from causal_self_attention_gqa_b200.workloads import (LAYER_WORKLOADS, LayerWorkload, Workload,
-                                                      make_layer_inputs)
+                                                      make_layer_inputs, packed_segment_ids)
 
 pytestmark = pytest.mark.gpu
 
@@ -177,10 +177,23 @@ def test_layer_matches_oracle(csa, case):
     B, T, C, Hq, Hkv, D, opts = case
     a = Workload("t", B=B, T=T, Hq=Hq, Hkv=Hkv, D=D, **opts)
     inp = make_layer_inputs(LayerWorkload("t", a, C=C, seed=B * T + C))
-    y, grads = _layer_gpu(csa, inp, a)
+    _check_layer(csa, a, inp, None)
+
+
+def test_layer_packed_segments(csa):
+    """The layer over packed rows: segment_ids restrict attention to each document and restart
+    the RoPE positions, inside the same projection -> attention -> projection step."""
+    a = Workload("t", B=2, T=400, Hq=4, Hkv=2, D=64, rope_base=10000.0, qk_norm=True, window=96)
+    inp = make_layer_inputs(LayerWorkload("t", a, C=256, seed=77))
+    seg = torch.from_numpy(packed_segment_ids(a.B, a.T, 20, 160, 77))
+    _check_layer(csa, a, inp, seg)
+
+
+def _check_layer(csa, a, inp, seg):
+    y, grads = _layer_gpu(csa, inp, a, None if seg is None else seg.to(DEV))
     ref_in = [inp[n].double().numpy() for n in ("x", "wq", "wk", "wv", "wo")]
-    ref_y, _ = proj.attn_layer_fwd(*ref_in, **a.options())
-    ref_g = proj.attn_layer_bwd(*ref_in, inp["dy"].double().numpy(), **a.options())
+    ref_y, _ = proj.attn_layer_fwd(*ref_in, segment_ids=seg, **a.options())
+    ref_g = proj.attn_layer_bwd(*ref_in, inp["dy"].double().numpy(), segment_ids=seg, **a.options())
     yn = _np(y)
     assert _rel(yn, ref_y) <= 1e-2 and float(np.max(np.abs(yn - ref_y))) <= 2e-2
     for got, ref, n in zip(grads, ref_g, ("dx", "dwq", "dwk", "dwv", "dwo")):
