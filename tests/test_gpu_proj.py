@@ -76,6 +76,9 @@ SHAPES = [
     (1, 18944, 640, 5, 5, 128),  # Q/K/V and dw 128-wide
     (1, 2048, 768, 8, 4, 96),    # y, dO, dx 128-wide
     (2, 4096, 640, 5, 5, 128),   # y, dO, dx 192-wide
+    # CTA pairs with a ragged last 256-row tile, an N tail (C = 320) and a 256-column tile that
+    # straddles all three Q/K/V pieces (320 / 64 / 64)
+    (1, 19044, 320, 5, 1, 64),
 ]
 
 
