@@ -16,8 +16,10 @@
 //             dwo  += o^T dy                A = o M-major,   B = dy N-major, fp32 out
 //             dwq|dwk|dwv += x^T [dq|dk|dv] A = x M-major,   B, C pieced by N, fp32 out
 //
-// Kernel: persistent (one CTA per SM, 192 threads), tiles of 128 x bn (bn up to 256), K in
-// blocks of 64 through a STAGES-deep shared-memory ring:
+// Two kernels, both persistent (one CTA per SM, 192 threads) with the same roles: k_gemm_pair
+// (below) runs large products on CTA pairs with 256 x 256 tiles; k_gemm runs the rest on
+// single CTAs.  k_gemm: tiles of 128 x bn (bn up to 256), K in blocks of 64 through a
+// STAGES-deep shared-memory ring:
 //   warp 0, one lane   TMA producer: the A tile (one 64 x 128 box K-major, or two 64 x 64
 //                      boxes M-major) and the B tile of the next K block, 128-byte swizzle;
 //   warp 1, one lane   tcgen05.mma issuer (M = 128, N = bn, K = 16 per instruction) into one

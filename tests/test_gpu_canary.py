@@ -77,3 +77,46 @@ def test_outputs_and_workspace_stay_in_bounds(csa, case, after_fwd):
     # the guarded outputs are the real results: finite everywhere
     for name, g in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
         assert torch.isfinite(g.t.float()).all(), name
+
+
+PROJ_CASES = [
+    # (B, T, C, Hq, Hkv, D): a single-CTA shape with a ragged 128-row tile, and a CTA-pair
+    # shape whose last 256-row tile and last 256-column tile are partly outside the tensors
+    (1, 300, 256, 4, 2, 64),
+    (1, 19044, 320, 5, 1, 64),
+]
+
+
+@pytest.mark.parametrize("case", PROJ_CASES, ids=lambda c: "B%dT%dC%dH%dx%dD%d" % c)
+def test_projection_outputs_stay_in_bounds(csa, case):
+    """The TMA stores (bf16 products) and reduce-adds (fp32 weight gradients) of the four
+    projection calls never write outside their tensors."""
+    B, T, C, Hq, Hkv, D = case
+    dev = torch.device("cuda:0")
+    g = torch.Generator().manual_seed(T)
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(dev)
+
+    x, dy = rnd(B, T, C), rnd(B, T, C)
+    wq, wk, wv = rnd(C, Hq, D, std=C ** -0.5), rnd(C, Hkv, D, std=C ** -0.5), rnd(C, Hkv, D, std=C ** -0.5)
+    wo = rnd(Hq, D, C, std=(Hq * D) ** -0.5)
+    o = rnd(B, T, Hq, D)
+    bf = torch.bfloat16
+    gq, gk, gv = (Guarded((B, T, H, D), bf, dev) for H in (Hq, Hkv, Hkv))
+    gy, gdx = Guarded((B, T, C), bf, dev), Guarded((B, T, C), bf, dev)
+    gdo = Guarded((B, T, Hq, D), bf, dev)
+    gdwo = Guarded((Hq, D, C), torch.float32, dev)
+    gdw = [Guarded((C, H, D), torch.float32, dev) for H in (Hq, Hkv, Hkv)]
+    for t in [gdwo] + gdw:
+        t.t.zero_()
+    csa.qkv_proj(x, wq, wk, wv, q=gq.t, k=gk.t, v=gv.t)
+    csa.out_proj(o, wo, y=gy.t)
+    csa.out_proj_bwd(o, wo, dy, dout=gdo.t, dwo=gdwo.t)
+    csa.qkv_proj_bwd(x, wq, wk, wv, gq.t, gk.t, gv.t, dx=gdx.t, dwq=gdw[0].t, dwk=gdw[1].t, dwv=gdw[2].t)
+    torch.cuda.synchronize()
+    for name, t in (("q", gq), ("k", gk), ("v", gv), ("y", gy), ("dout", gdo), ("dx", gdx), ("dwo", gdwo),
+                    ("dwq", gdw[0]), ("dwk", gdw[1]), ("dwv", gdw[2])):
+        assert t.intact(), name
+    # and the products are there (not a silent no-op)
+    assert float(gq.t.float().abs().sum()) > 0 and float(gdw[2].t.abs().sum()) > 0
