@@ -35,6 +35,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "csa_internal.h"
 #include "ptx.cuh"
 
@@ -553,13 +555,23 @@ cudaError_t launch_pair_t(const GemmMaps& maps, const GemmArgs& g, cudaStream_t 
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // as many pairs as can be resident at once (clusters are placed within a GPC)
-    int clusters = 0;
-    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-    e = cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg);
-    if (e != cudaSuccess || clusters < 1) {
+    // as many pairs as can be resident at once (clusters are placed within a GPC); asked of
+    // the runtime once per device for each of the three kernels
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
-        clusters = num_sms() / 2;
+        dev = -1;
+    }
+    static std::atomic<int> resident[64];  // 0: not asked yet (zero-initialised, static storage)
+    int clusters = dev >= 0 ? resident[dev].load(std::memory_order_relaxed) : 0;
+    if (clusters < 1) {
+        cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+        e = cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg);
+        if (e != cudaSuccess || clusters < 1) {
+            cudaGetLastError();
+            clusters = num_sms() / 2;
+        }
+        if (dev >= 0) resident[dev].store(clusters, std::memory_order_relaxed);
     }
     const int npairs = g.units < clusters ? g.units : clusters;
     cfg.gridDim = dim3(2 * npairs, 1, 1);
