@@ -590,8 +590,8 @@ int pick_bn(const int* widths, int npieces, int M, bool split_k) {
 // (split_k) cut K so that about one unit runs per SM (per CTA pair), keeping at least 4 K
 // blocks a split.  Large products run on CTA pairs (256 x 256 tiles, cta_group::2) when
 // allow_pair: at least one unit for every pair of SMs.  A K-major B with several N pieces
-// cannot (its 128-column half-box would straddle them); the callers pass allow_pair = false
-// there.
+// never does (its 128-column half-box would straddle them).  The operand forms (a_mn, b_mn,
+// b_by_k) must be set in g before the call.
 void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const int* kw, int nk, bool split_k,
                bool allow_pair, int* status) {
     g.M = M;
@@ -605,6 +605,8 @@ void plan_gemm(GemmArgs& g, int M, int N, int K, const int* nw, int nn, const in
     g.kb_total = (K + 63) / 64;
     g.status = status;
     const int pairs = num_sms() / 2;
+    // a K-major B is loaded as one 128-column half-box per CTA, which must not straddle N pieces
+    if (!g.b_mn && !g.b_by_k && nn > 1) allow_pair = false;
     if (allow_pair) {
         const int mt2 = (M + 255) / 256, nt2 = (N + 255) / 256;
         int splits = 1;
