@@ -72,6 +72,61 @@ __device__ __forceinline__ int piece(const int (&bound)[4], int x) {
     return (x >= bound[1]) + (x >= bound[2]);
 }
 
+// One epilogue chunk of one warp: 32 accumulator rows (this warp's TMEM lane quarter, from
+// column address `tcol`) x 32 fp32 or 64 bf16 columns -> one 32 x 128-byte staging box in
+// the TMA box layout (128-byte swizzle: 16-byte chunk j of row r at j ^ (r & 7)) -> a TMA
+// reduce-add (fp32) or store (bf16) at (column, row) of `map`.  `nst` counts this warp's
+// chunks so far; the two boxes alternate, and a box is rewritten only once the store that
+// last read it has finished reading.  Every lane of the warp calls it.
+template <bool F32>
+__device__ __forceinline__ void epilogue_chunk(uint32_t tcol, uint8_t* stg, int nst, const CUtensorMap* map,
+                                               int column, int row) {
+    const int lane = threadIdx.x & 31, sw = lane & 7;
+    uint8_t* box = stg + (nst & 1) * 4096;
+    if (lane == 0 && nst >= 2) bulk_wait_group_read1();
+    __syncwarp();
+    if (F32) {
+        uint32_t v[32];
+        tmem_ld32(tcol, v);
+        tmem_ld_wait();
+        tmem_ld_fence(v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) =
+                make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tcol, v0);
+        tmem_ld32(tcol + 32, v1);
+        tmem_ld_wait();
+        tmem_ld_fence(v0);
+        tmem_ld_fence(v1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) = make_uint4(
+                pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
+                pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
+                pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
+                pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(box + lane * 128 + (((j + 4) ^ sw) * 16)) = make_uint4(
+                pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
+                pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
+                pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
+                pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        if (F32)
+            tma_reduce_add_2d(map, box, column, row);
+        else
+            tma_store_2d(map, box, column, row);
+        bulk_commit_group();
+    }
+}
+
 template <int BN, bool A_MN, bool B_MN, bool F32>
 __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs g) {
     using C = GemmCfg<BN, F32>;
@@ -195,7 +250,6 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ GemmMap
     } else {
         const int quarter = warp & 3;  // the TMEM lanes (tile rows) this warp may read
         uint8_t* stg = smem + C::OFF_STG + (warp - 2) * C::STG_WARP;
-        const int sw = lane & 7;
         int t = 0, nst = 0;
         for (int u = blockIdx.x; u < g.units; u += gridDim.x, ++t) {
             int m0, n0, kb0, kb1;
@@ -209,52 +263,8 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ GemmMap
             const uint32_t ta = tmem + ((uint32_t)(32 * quarter) << 16) + buf * C::ACC;
             const int row0 = m0 + 32 * quarter;
 #pragma unroll 1
-            for (int c = 0; c < BN / C::CHUNK; ++c, ++nst) {
-                uint8_t* box = stg + (nst & 1) * 4096;
-                // the previous store out of this box has finished reading it
-                if (lane == 0 && nst >= 2) bulk_wait_group_read1();
-                __syncwarp();
-                if (F32) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + 32 * c, v);
-                    tmem_ld_wait();
-                    tmem_ld_fence(v);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) =
-                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                } else {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(ta + 64 * c, v0);
-                    tmem_ld32(ta + 64 * c + 32, v1);
-                    tmem_ld_wait();
-                    tmem_ld_fence(v0);
-                    tmem_ld_fence(v1);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + (((j + 4) ^ sw) * 16)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (F32)
-                        tma_reduce_add_2d(mc, box, nl + C::CHUNK * c, row0);
-                    else
-                        tma_store_2d(mc, box, nl + C::CHUNK * c, row0);
-                    bulk_commit_group();
-                }
-            }
+            for (int c = 0; c < BN / C::CHUNK; ++c, ++nst)
+                epilogue_chunk<F32>(ta + C::CHUNK * c, stg, nst, mc, nl + C::CHUNK * c, row0);
             // every column of this accumulator is in registers or staged: the MMAs may reuse it
             tc_fence_before();
             warp_arrive(&acc_empty[buf]);
@@ -452,7 +462,6 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         const int quarter = warp & 3;
         uint8_t* stg = smem + C::OFF_STG + (warp - 2) * C::STG_WARP;
-        const int sw = lane & 7;
         const uint32_t acc_empty0 = mapa_shared(smem_u32(&acc_empty[0]), 0);  // the leader's
         int t = 0, nst = 0;
         for (int u = pair_id; u < g.units; u += npairs, ++t) {
@@ -468,51 +477,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int n = n0 + C::CHUNK * c;
                 if (n >= g.N) break;  // warp-uniform; columns past N are never stored
                 const int np = piece(g.n_bound, n);
-                const CUtensorMap* mc = &maps.c[np];
-                uint8_t* box = stg + (nst & 1) * 4096;
-                if (lane == 0 && nst >= 2) bulk_wait_group_read1();
-                __syncwarp();
-                if (F32) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + 32 * c, v);
-                    tmem_ld_wait();
-                    tmem_ld_fence(v);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) =
-                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                } else {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(ta + 64 * c, v0);
-                    tmem_ld32(ta + 64 * c + 32, v1);
-                    tmem_ld_wait();
-                    tmem_ld_fence(v0);
-                    tmem_ld_fence(v1);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ sw) * 16)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v0[8 * j]), __uint_as_float(v0[8 * j + 1])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 2]), __uint_as_float(v0[8 * j + 3])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 4]), __uint_as_float(v0[8 * j + 5])),
-                            pack_bf16x2(__uint_as_float(v0[8 * j + 6]), __uint_as_float(v0[8 * j + 7])));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(box + lane * 128 + (((j + 4) ^ sw) * 16)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v1[8 * j]), __uint_as_float(v1[8 * j + 1])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 2]), __uint_as_float(v1[8 * j + 3])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 4]), __uint_as_float(v1[8 * j + 5])),
-                            pack_bf16x2(__uint_as_float(v1[8 * j + 6]), __uint_as_float(v1[8 * j + 7])));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (F32)
-                        tma_reduce_add_2d(mc, box, n - g.n_bound[np], row0);
-                    else
-                        tma_store_2d(mc, box, n - g.n_bound[np], row0);
-                    bulk_commit_group();
-                }
-                ++nst;
+                epilogue_chunk<F32>(ta + C::CHUNK * c, stg, nst++, &maps.c[np], n - g.n_bound[np], row0);
             }
             // this CTA's half is out of TMEM: tell the leader's MMA thread
             tc_fence_before();
